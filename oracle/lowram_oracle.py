@@ -1,0 +1,261 @@
+"""Oracle: the plain, slow fp64 reference of LowRAM's compressed-cache path.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this module. The product path (the
+CUDA library and its Python binding) never calls it, and this module imports
+nothing from the product. The two share only the seeded input generator.
+
+Every function is the plain definition of one step, written in fp64 numpy with
+library primitives (matmul, erf, a stable sort) and no blocking, fusion or
+reordering. Inputs are taken as the exact values of the storage type (bf16 or
+fp32 values held in float64). Sources, by page and section:
+
+* "LowRAM" project page, Figure 3 ("Store the pattern, keep the exceptions"):
+  the keys of a group of adjacent layers share one per-token factor A and each
+  layer keeps its own smaller factor, K ~= A.B.
+* "LowRAM KV cache compression -- Predicting the value cache from keys"
+  (explainer), paragraph 2: values are rebuilt as the predictor's output plus
+  an exact residual where one is stored, then used by ordinary attention;
+  paragraph 3: the predictor starts from the pseudoinverse linear map and adds a
+  small nonlinear branch; paragraph 4: residuals go to the tokens ranked worst
+  by reconstruction error, one predictor per head; the "Where the memory
+  actually goes" paragraph: the per-head storage budget.
+* arXiv 2611.07025 abstract page: only a selected subset of the cached pairs
+  is rebuilt at each decoding step (selective reconstruction).
+
+Readings where the pages are silent (each also listed in the design notes):
+the predictor sees the reconstructed key; a residual is the difference
+``v - v_hat``; the error is the squared L2 norm over the head's entries; ties
+in the error ranking go to the lower token index; GELU is the exact erf form;
+the softmax scale is ``1/sqrt(head_dim)``; an empty attention set gives a zero
+output; the stored factor A and residual rows are rounded to the storage type
+with round-to-nearest-even.
+
+Parity pins: every function here is checked by ``tests/test_oracle_pins.py``
+against facts the pages or mathematics fix (Slim-Attention exactness, 100 %
+residual budget, full-rank keys, brute-force top-k, tabulated normal CDF
+values, a hand-computed predictor, the worked memory example).
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+from scipy.special import erf
+
+BLOCK = 64
+
+
+# --------------------------------------------------------------------------- storage rounding
+
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (ties to even), returned as fp64.
+
+    bfloat16 keeps 8 significant bits and the fp32 exponent range: a normal
+    value in [2^e, 2^(e+1)) is rounded to a multiple of 2^(e-7); below 2^-126
+    the spacing stays 2^-133. Overflow past the largest finite value gives inf.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, dtype=np.float64, copy=True)
+    fin = np.isfinite(x) & (x != 0)
+    xf = x[fin]
+    _, e = np.frexp(np.abs(xf))          # |x| = m * 2^e, m in [0.5, 1): |x| in [2^(e-1), 2^e)
+    q = np.ldexp(1.0, np.maximum(e - 1 - 7, -133))   # spacing of bf16 values in that binade
+    r = np.round(xf / q) * q             # np.round: half to even; xf/q is exact (power of two)
+    big = np.abs(r) >= 2.0 ** 128
+    r[big] = np.copysign(np.inf, r[big])
+    out[fin] = r
+    return out
+
+
+def round_storage(x, dtype: str) -> np.ndarray:
+    """Round to the storage type named by dtype ('f64' keeps values, 'f32', 'bf16')."""
+    x = np.asarray(x, dtype=np.float64)
+    if dtype == "f64":
+        return x.copy()
+    if dtype == "f32":
+        return x.astype(np.float32).astype(np.float64)
+    if dtype == "bf16":
+        return round_bf16(x)
+    raise ValueError(dtype)
+
+
+# --------------------------------------------------------------------------- method steps
+
+def gelu(x) -> np.ndarray:
+    """GELU, exact form: x * Phi(x) = 0.5 x (1 + erf(x / sqrt 2))."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def project_keys(K_group: np.ndarray, Bt: np.ndarray) -> np.ndarray:
+    """Shared factor A = K_group . B^T for one sequence (project page, Figure 3).
+
+    K_group [T, D] holds the concatenated keys of the layer group; Bt [D, r]
+    holds the basis B^T whose columns are orthonormal (a truncated SVD's right
+    singular vectors), so A is the least-squares coefficient matrix of K on B.
+    """
+    return np.asarray(K_group, np.float64) @ np.asarray(Bt, np.float64)
+
+
+def key_slice(Bt: np.ndarray, layer: int, head: int, n_kv_heads: int, head_dim: int) -> np.ndarray:
+    """B_l^h as rows of Bt: [hd, r], the basis rows belonging to (layer, KV head)."""
+    c0 = (layer * n_kv_heads + head) * head_dim
+    return np.asarray(Bt, np.float64)[c0:c0 + head_dim, :]
+
+
+def reconstruct_keys(A: np.ndarray, Bt_lh: np.ndarray) -> np.ndarray:
+    """k~_t = A[t] . B_l^h for every row of A (project page, Figure 3)."""
+    return np.asarray(A, np.float64) @ np.asarray(Bt_lh, np.float64).T
+
+
+def predict_values(kt, W_lin, W1, b1, W2, b2=None) -> np.ndarray:
+    """v_hat = k~ W_lin^T + GELU(k~ W1^T + b1) W2^T + b2 (explainer, paragraphs 2-3).
+
+    Weights are in nn.Linear layout (out x in): W_lin [hd, hd], W1 [H, hd],
+    b1 [H], W2 [hd, H], b2 [hd] (None means zero).
+    """
+    kt = np.asarray(kt, np.float64)
+    u = kt @ np.asarray(W1, np.float64).T + np.asarray(b1, np.float64)
+    v = kt @ np.asarray(W_lin, np.float64).T + gelu(u) @ np.asarray(W2, np.float64).T
+    if b2 is not None:
+        v = v + np.asarray(b2, np.float64)
+    return v
+
+
+def token_errors(v, v_hat) -> np.ndarray:
+    """e_t = sum_j (v_t[j] - v_hat_t[j])^2: squared L2 error per token (explainer, paragraph 4)."""
+    d = np.asarray(v, np.float64) - np.asarray(v_hat, np.float64)
+    return np.sum(d * d, axis=-1)
+
+
+def topk_residual_tokens(e, k: int) -> np.ndarray:
+    """The k tokens with the largest error, ties to the lower index, returned ascending.
+
+    Orders tokens by (error descending, index ascending), keeps the first k and
+    sorts those indices (explainer, paragraph 4: residuals go to the worst tokens).
+    """
+    e = np.asarray(e, np.float64)
+    T = e.shape[0]
+    if not 0 <= k <= T:
+        raise ValueError("k out of range")
+    order = np.lexsort((np.arange(T), -e))
+    return np.sort(order[:k]).astype(np.int64)
+
+
+def block_ptr(idx, T: int, block: int = BLOCK) -> np.ndarray:
+    """ptr[j] = number of residual indices below block * j, for j = 0 .. ceil(T/block)."""
+    idx = np.asarray(idx, np.int64)
+    nblk = (T + block - 1) // block
+    return np.array([int(np.count_nonzero(idx < block * j)) for j in range(nblk + 1)], dtype=np.int64)
+
+
+def pack_sequence(K_group, V, Bt, W_lin, W1, b1, W2, b2, k: int, dtype: str,
+                  n_kv_heads: int, head_dim: int) -> Dict[str, np.ndarray]:
+    """The prefill-side packer for one sequence, step by step.
+
+    K_group [T, D]; V [L, T, Hkv, hd]; Bt [D, r]; predictor arrays indexed
+    [L, Hkv, ...]. Returns A (rounded to dtype), idx [L, Hkv, k] ascending,
+    val [L, Hkv, k, hd] (rounded), ptr [L, Hkv, nblk+1] and err [L, Hkv, T].
+    """
+    A = round_storage(project_keys(K_group, Bt), dtype)
+    L, T = V.shape[0], V.shape[1]
+    nblk = (T + BLOCK - 1) // BLOCK
+    idx = np.zeros((L, n_kv_heads, k), np.int64)
+    val = np.zeros((L, n_kv_heads, k, head_dim), np.float64)
+    ptr = np.zeros((L, n_kv_heads, nblk + 1), np.int64)
+    err = np.zeros((L, n_kv_heads, T), np.float64)
+    for l in range(L):
+        for h in range(n_kv_heads):
+            kt = reconstruct_keys(A, key_slice(Bt, l, h, n_kv_heads, head_dim))
+            vh = predict_values(kt, W_lin[l, h], W1[l, h], b1[l, h], W2[l, h],
+                                None if b2 is None else b2[l, h])
+            v = np.asarray(V[l, :, h, :], np.float64)
+            e = token_errors(v, vh)
+            sel = topk_residual_tokens(e, k)
+            err[l, h] = e
+            idx[l, h] = sel
+            val[l, h] = round_storage(v[sel] - vh[sel], dtype)
+            ptr[l, h] = block_ptr(sel, T)
+    return {"A": A, "idx": idx, "val": val, "ptr": ptr, "err": err}
+
+
+def selected_tokens(T: int, blocks: Optional[Sequence[int]], block: int = BLOCK) -> np.ndarray:
+    """Token indices attended: all of [0, T) (blocks None), else the union of the blocks' ranges."""
+    if blocks is None:
+        return np.arange(T, dtype=np.int64)
+    parts = [np.arange(block * j, min(block * j + block, T), dtype=np.int64) for j in blocks]
+    if not parts:
+        return np.zeros(0, np.int64)
+    return np.unique(np.concatenate(parts))
+
+
+def decode_sequence(q, A, Bt, W_lin, W1, b1, W2, b2, layer: int, res_idx, res_val,
+                    blocks, scale: float, n_kv_heads: int, head_dim: int) -> np.ndarray:
+    """One decode step of one layer for one sequence: o [Hq, hd].
+
+    For KV head h: gather the attended tokens (all, or the selected blocks:
+    arXiv abstract, selective reconstruction), rebuild their keys A.B_l^h,
+    rebuild their values as prediction + residual where one is stored
+    (explainer, paragraph 2), and run softmax attention for the query heads
+    h*G .. h*G+G-1 with max-subtracted exponentials. Predictor arrays are
+    indexed [L, Hkv, ...]; res_idx [L, Hkv, k]; res_val [L, Hkv, k, hd];
+    blocks is None (all tokens) or a per-KV-head sequence of block ids.
+    """
+    q = np.asarray(q, np.float64)
+    Hq = q.shape[0]
+    G = Hq // n_kv_heads
+    T = A.shape[0]
+    o = np.zeros((Hq, head_dim), np.float64)
+    for h in range(n_kv_heads):
+        S = selected_tokens(T, None if blocks is None else blocks[h])
+        if S.size == 0:
+            continue
+        kt = reconstruct_keys(np.asarray(A, np.float64)[S], key_slice(Bt, layer, h, n_kv_heads, head_dim))
+        v = predict_values(kt, W_lin[layer, h], W1[layer, h], b1[layer, h], W2[layer, h],
+                           None if b2 is None else b2[layer, h])
+        r_full = np.zeros((T, head_dim), np.float64)
+        r_full[np.asarray(res_idx[layer, h], np.int64)] = np.asarray(res_val[layer, h], np.float64)
+        v = v + r_full[S]
+        for g in range(G):
+            hq = h * G + g
+            s = (kt @ q[hq]) * scale
+            w = np.exp(s - s.max())
+            o[hq] = (w @ v) / w.sum()
+    return o
+
+
+def default_scale(head_dim: int, scale: float) -> float:
+    """The softmax scale: the given one when positive, else 1/sqrt(head_dim)."""
+    return scale if scale > 0 else 1.0 / math.sqrt(head_dim)
+
+
+def dense_attention(q, K, V, scale: float) -> np.ndarray:
+    """Textbook single-query attention: softmax(q K^T * scale) V, for q [hd], K, V [T, hd]."""
+    s = (np.asarray(K, np.float64) @ np.asarray(q, np.float64)) * scale
+    w = np.exp(s - s.max())
+    return (w @ np.asarray(V, np.float64)) / w.sum()
+
+
+# --------------------------------------------------------------------------- accounting
+
+def predictor_numbers(head_dim: int, hidden: int) -> int:
+    """Stored numbers of one head's predictor: W_lin, W1, W2 and the two bias vectors."""
+    return head_dim * head_dim + 2 * head_dim * hidden + hidden + head_dim
+
+
+def residual_budget(T: int, head_dim: int, ratio: float, hidden: int) -> float:
+    """Residual rows one head can afford at a target value-cache compression ratio.
+
+    Follows the explainer's "Where the memory actually goes" paragraph: the
+    head's value cache holds T*hd numbers, the target keeps T*hd/ratio of them,
+    the predictor is a fixed cost, and each residual costs hd numbers plus an
+    index counted as two numbers.
+    """
+    return (T * head_dim / ratio - predictor_numbers(head_dim, hidden)) / (head_dim + 2)
+
+
+def dense_cache_bytes_per_token(n_layers: int, n_kv_heads: int, head_dim: int, elem_bytes: int) -> int:
+    """Bytes one token adds to an uncompressed K+V cache."""
+    return n_layers * n_kv_heads * head_dim * 2 * elem_bytes

@@ -1,0 +1,286 @@
+"""Pins of the oracle against facts the pages and mathematics fix (CPU only).
+
+Each test is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign, index or head slice, a transposed weight, the tanh GELU instead of
+the erf form) fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lowram_oracle as orc
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _orthogonal(rng, n):
+    q, r = np.linalg.qr(rng.standard_normal((n, n)))
+    return q * np.sign(np.diag(r))
+
+
+# ----------------------------------------------------------------------------- rounding
+
+def test_round_bf16_ties_and_torch():
+    r = orc.round_bf16
+    assert r(1.0) == 1.0
+    assert r(1.0 + 2.0 ** -8) == 1.0                      # tie -> even (1.0)
+    assert r(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6      # tie -> even (mantissa ...10)
+    assert r(1.0 + 2.0 ** -8 + 2.0 ** -20) == 1.0 + 2.0 ** -7
+    assert r(-3.0) == -3.0 and r(0.0) == 0.0
+    assert np.isinf(r(3.5e38))
+    rng = np.random.default_rng(0)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.round_bf16(x.astype(np.float64)), ref)
+
+
+# ----------------------------------------------------------------------------- GELU
+
+def test_gelu_is_exact_erf_form():
+    for x, phi in _gold("normal_cdf.json")["values"]:
+        assert abs(orc.gelu(x) - x * phi) <= 1e-12 * max(1.0, abs(x))
+    # the tanh approximation differs by ~1.6e-4 at x = 1; the pin above rejects it
+    tanh_form = 0.5 * (1 + math.tanh(math.sqrt(2 / math.pi) * (1 + 0.044715)))
+    assert abs(tanh_form - orc.gelu(1.0)) > 1e-5
+
+
+# ----------------------------------------------------------------------------- predictor
+
+def test_predict_values_hand_computed():
+    # k = [1, -1]; W_lin (out x in) = [[1, 2], [0, 1]] -> k W_lin^T = [1*1 + 2*-1, 0*1 + 1*-1] = [-1, -1]
+    # u = k W1^T + b1 with W1 = I, b1 = [0, 0.5] -> [1, -0.5]; g = [Phi(1), -0.5 Phi(-0.5)]
+    # W2 (out x in) = [[2, 5], [0, 3]] -> g W2^T = [2 g0 + 5 g1, 3 g1]; b2 = [0.5, -1]
+    phi1 = 0.8413447460685429
+    phim05 = 1.0 - 0.6914624612740131
+    g0, g1 = 1.0 * phi1, -0.5 * phim05
+    expect = np.array([-1 + 2 * g0 + 5 * g1 + 0.5, -1 + 3 * g1 - 1.0])
+    got = orc.predict_values(np.array([[1.0, -1.0]]), np.array([[1.0, 2.0], [0.0, 1.0]]),
+                             np.eye(2), np.array([0.0, 0.5]), np.array([[2.0, 5.0], [0.0, 3.0]]),
+                             np.array([0.5, -1.0]))
+    np.testing.assert_allclose(got[0], expect, rtol=0, atol=1e-12)
+
+
+def test_token_errors_squared_l2():
+    v = np.array([[3.0, 4.0, 1.0], [0.0, 0.0, 0.0]])
+    vh = np.array([[0.0, 0.0, 1.0], [1.0, -2.0, 2.0]])
+    np.testing.assert_array_equal(orc.token_errors(v, vh), [25.0, 9.0])
+
+
+# ----------------------------------------------------------------------------- top-k
+
+def _unique_valid_set(e, k):
+    """The one k-subset whose every member ranks above every non-member by (e desc, t asc)."""
+    T = len(e)
+    found = []
+    for S in itertools.combinations(range(T), k):
+        s = set(S)
+        ok = all((e[i] > e[j]) or (e[i] == e[j] and i < j)
+                 for i in s for j in range(T) if j not in s)
+        if ok:
+            found.append(S)
+    assert len(found) == 1
+    return np.array(found[0], dtype=np.int64)
+
+
+@pytest.mark.parametrize("ties", [False, True])
+def test_topk_matches_brute_force(ties):
+    rng = np.random.default_rng(7 if ties else 3)
+    for T in range(0, 11):
+        for trial in range(3):
+            e = (rng.integers(0, 3, T).astype(float) if ties else rng.random(T))
+            for k in range(0, T + 1):
+                got = orc.topk_residual_tokens(e, k)
+                np.testing.assert_array_equal(got, _unique_valid_set(e, k))
+                # the set minimises the error left uncorrected over all k-subsets
+                left = e.sum() - e[got].sum()
+                best = min((e.sum() - sum(e[list(S)]) for S in itertools.combinations(range(T), k)),
+                           default=0.0)
+                assert abs(left - best) <= 1e-12
+
+
+def test_topk_remaining_error_invariant_large():
+    rng = np.random.default_rng(11)
+    e = rng.random(5000) ** 3
+    k = 731
+    sel = orc.topk_residual_tokens(e, k)
+    left = np.delete(e, sel).sum()
+    assert abs(left - np.sort(e)[: 5000 - k].sum()) <= 1e-9
+    for _ in range(20):
+        rnd = rng.choice(5000, k, replace=False)
+        assert left <= np.delete(e, rnd).sum()
+    assert np.all(np.diff(sel) > 0)
+
+
+def test_block_ptr_properties():
+    rng = np.random.default_rng(5)
+    for T in (1, 63, 64, 65, 1000, 4097):
+        for k in (0, 1, min(T, 17), T):
+            idx = np.sort(rng.choice(T, k, replace=False))
+            ptr = orc.block_ptr(idx, T)
+            nblk = (T + 63) // 64
+            assert len(ptr) == nblk + 1 and ptr[0] == 0 and ptr[-1] == k
+            for j in range(nblk):
+                seg = idx[ptr[j]:ptr[j + 1]]
+                assert np.all((seg >= 64 * j) & (seg < 64 * j + 64))
+
+
+# ----------------------------------------------------------------------------- attention pins
+
+def test_dense_attention_hand():
+    q = np.array([1.0, 0.0])
+    K = np.array([[1.0, 0.0], [0.0, 1.0]])
+    V = np.array([[2.0, 0.0], [0.0, 4.0]])
+    p0 = math.e / (math.e + 1)
+    np.testing.assert_allclose(orc.dense_attention(q, K, V, 1.0), [2 * p0, 4 * (1 - p0)], atol=1e-14)
+    np.testing.assert_allclose(orc.dense_attention(q, K[:1], V[:1], 0.3), V[0], atol=1e-15)
+    np.testing.assert_allclose(orc.dense_attention(np.zeros(2), K, V, 1.0), V.mean(0), atol=1e-15)
+    assert orc.default_scale(64, 0.0) == 0.125 and orc.default_scale(64, 0.5) == 0.5
+
+
+def _hidden(rng, T, d):
+    return rng.standard_normal((T, d))
+
+
+def test_slim_attention_exact_recovery():
+    """Square invertible key projection, zero nonlinear branch: v_hat = v and o = dense attention."""
+    rng = np.random.default_rng(21)
+    d = hd = 64
+    T, G = 300, 2
+    W_K = _orthogonal(rng, d) @ np.diag(np.linspace(0.5, 2.0, d))
+    W_V = rng.standard_normal((d, hd)) / 8
+    W_Q = rng.standard_normal((d, G * hd)) / 8
+    x = _hidden(rng, T, d)
+    K, V = x @ W_K, x @ W_V
+    Bt = _orthogonal(rng, d)                      # full-rank basis (r = D)
+    W_lin = (np.linalg.pinv(W_K) @ W_V).T[None, None]
+    W1 = rng.standard_normal((1, 1, 32, hd)) * 0.1
+    b1 = rng.standard_normal((1, 1, 32))
+    W2 = np.zeros((1, 1, hd, 32))
+    packed = orc.pack_sequence(K, V[None, :, None, :], Bt, W_lin, W1, b1, W2, None, 0, "f64", 1, hd)
+    assert packed["err"].max() <= 1e-18 * np.sum(V * V)
+    q = (rng.standard_normal((1, d)) @ W_Q).reshape(G, hd)
+    o = orc.decode_sequence(q, packed["A"], Bt, W_lin, W1, b1, W2, None, 0, packed["idx"],
+                            packed["val"], None, orc.default_scale(hd, 0), 1, hd)
+    for g in range(G):
+        ref = orc.dense_attention(q[g], K, V, 1 / math.sqrt(hd))
+        np.testing.assert_allclose(o[g], ref, rtol=1e-10, atol=1e-10 * np.abs(ref).max())
+
+
+def _group_problem(rng, d=64, L=2, Hkv=2, G=2, hd=16, T=200, H=24):
+    WK = rng.standard_normal((L, d, Hkv * hd)) / 8
+    WV = rng.standard_normal((L, d, Hkv * hd)) / 8
+    x = _hidden(rng, T, d)
+    K_group = np.concatenate([x @ WK[l] for l in range(L)], axis=1)     # [T, D]
+    V = np.stack([(x @ WV[l]).reshape(T, Hkv, hd) for l in range(L)])   # [L, T, Hkv, hd]
+    pred = dict(W_lin=rng.standard_normal((L, Hkv, hd, hd)) * 0.3,
+                W1=rng.standard_normal((L, Hkv, H, hd)) * 0.3,
+                b1=rng.standard_normal((L, Hkv, H)),
+                W2=rng.standard_normal((L, Hkv, hd, H)) * 0.3,
+                b2=rng.standard_normal((L, Hkv, hd)))
+    return K_group, V, pred
+
+
+def test_full_rank_keys_reproduce_every_head_slice():
+    rng = np.random.default_rng(8)
+    L, Hkv, hd = 2, 2, 16
+    K_group, _, _ = _group_problem(rng, L=L, Hkv=Hkv, hd=hd)
+    Bt = _orthogonal(rng, K_group.shape[1])
+    A = orc.project_keys(K_group, Bt)
+    for l in range(L):
+        for h in range(Hkv):
+            kt = orc.reconstruct_keys(A, orc.key_slice(Bt, l, h, Hkv, hd))
+            c0 = (l * Hkv + h) * hd
+            np.testing.assert_allclose(kt, K_group[:, c0:c0 + hd], atol=1e-12)
+
+
+@pytest.mark.parametrize("selective", [False, True])
+def test_full_budget_reproduces_dense_attention(selective):
+    """k = T residuals and a full-rank key factor: o = dense attention over (K, V), any predictor."""
+    rng = np.random.default_rng(31 + selective)
+    L, Hkv, G, hd, T = 2, 2, 2, 16, 200
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])
+    packed = orc.pack_sequence(K_group, V, Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"],
+                               pred["b2"], T, "f64", Hkv, hd)
+    np.testing.assert_array_equal(packed["idx"][0, 0], np.arange(T))
+    blocks = [[0, 3], [1, 2, 3]] if selective else None
+    for layer in range(L):
+        q = rng.standard_normal((Hkv * G, hd))
+        o = orc.decode_sequence(q, packed["A"], Bt, pred["W_lin"], pred["W1"], pred["b1"],
+                                pred["W2"], pred["b2"], layer, packed["idx"], packed["val"],
+                                blocks, 0.0 + 0.2, Hkv, hd)
+        for hq in range(Hkv * G):
+            h = hq // G
+            S = orc.selected_tokens(T, None if blocks is None else blocks[h])
+            c0 = (layer * Hkv + h) * hd
+            ref = orc.dense_attention(q[hq], K_group[S, c0:c0 + hd], V[layer][S, h], 0.2)
+            np.testing.assert_allclose(o[hq], ref, rtol=1e-10, atol=1e-10)
+
+
+def test_selection_all_blocks_equals_full_and_empty_is_zero():
+    rng = np.random.default_rng(4)
+    L, Hkv, G, hd, T = 1, 2, 2, 16, 150
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])[:, :20]
+    packed = orc.pack_sequence(K_group, V, Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"],
+                               pred["b2"], 30, "bf16", Hkv, hd)
+    q = rng.standard_normal((Hkv * G, hd))
+    args = (packed["A"], Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"], pred["b2"], 0,
+            packed["idx"], packed["val"])
+    full = orc.decode_sequence(q, *args, None, 0.25, Hkv, hd)
+    allb = orc.decode_sequence(q, *args, [[0, 1, 2], [0, 1, 2]], 0.25, Hkv, hd)
+    np.testing.assert_allclose(full, allb, rtol=1e-13, atol=1e-13)
+    empty = orc.decode_sequence(q, *args, [[], [1]], 0.25, Hkv, hd)
+    assert np.all(empty[:G] == 0) and np.all(np.isfinite(empty[G:]))
+
+
+def test_residuals_are_value_minus_prediction_at_worst_tokens():
+    rng = np.random.default_rng(9)
+    L, Hkv, hd, T, k = 1, 1, 16, 120, 13
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])[:, :10]
+    p = orc.pack_sequence(K_group, V, Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"],
+                          pred["b2"], k, "f64", Hkv, hd)
+    kt = orc.reconstruct_keys(p["A"], orc.key_slice(Bt, 0, 0, Hkv, hd))
+    vh = orc.predict_values(kt, pred["W_lin"][0, 0], pred["W1"][0, 0], pred["b1"][0, 0],
+                            pred["W2"][0, 0], pred["b2"][0, 0])
+    e = ((V[0, :, 0] - vh) ** 2).sum(1)
+    worst = np.argsort(-e, kind="stable")[:k]
+    np.testing.assert_array_equal(p["idx"][0, 0], np.sort(worst))
+    np.testing.assert_allclose(p["val"][0, 0], (V[0, :, 0] - vh)[np.sort(worst)], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- accounting pins
+
+def test_worked_memory_example():
+    g = _gold("worked_memory_example.json")
+    hd, H, ratio = g["head_dim"], g["hidden"], g["ratio"]
+    assert orc.predictor_numbers(hd, H) == g["cases"][0]["predictor_numbers"]
+    c0, c1, c2 = g["cases"]
+    n0 = orc.residual_budget(c0["T"], hd, ratio, H)
+    assert c0["T"] * hd == c0["value_numbers"] and c0["T"] * hd // ratio == c0["budget_numbers"]
+    assert c0["budget_numbers"] - c0["predictor_numbers"] == c0["remaining_numbers"]
+    assert hd + 2 == c0["numbers_per_residual"]
+    assert round(n0) == c0["residuals_printed_approx"]
+    assert round(100 * n0 / c0["T"]) == c0["fraction_printed_approx_pct"]
+    n1 = orc.residual_budget(c1["T"], hd, ratio, H)
+    assert round(n1) == c1["residuals_printed_approx"]
+    assert round(100 * n1 / c1["T"]) == c1["fraction_printed_approx_pct"]
+    share = orc.predictor_numbers(hd, H) / (c2["T"] * hd / ratio)
+    assert abs(share - c2["predictor_share_approx"]) < 0.01
+
+
+def test_dense_cache_bytes():
+    g = _gold("dense_cache_size.json")
+    b = orc.dense_cache_bytes_per_token(g["n_layers"], g["n_kv_heads"], g["head_dim"], g["elem_bytes"])
+    assert round(b / 1000, 2) == g["kb_per_token_printed"]
