@@ -1,0 +1,442 @@
+#!/usr/bin/env python3
+"""Benchmark of the LowRAM compressed-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lowram|reference] [--workload NAME]
+
+A step is one lr_decode_attn call: one decode step of one layer over the whole
+compressed cache of the workload (B sequences of T tokens). The cache is built
+first by lr_pack_prefill from synthetic Mistral-7B-shaped keys and values (the
+packer's own timing is reported under "pack"). Steps cycle over the 4 layers of
+the group and over 4 device copies of the cache (more than twice the 126 MB L2),
+so no step finds its inputs in L2. With N GPUs (torchrun) every rank decodes its
+own sequences (weak scaling, no collective on the data path); the time is the
+maximum over ranks.
+
+The metric is context tokens per second per layer, B*T / (time of one layer's
+decode step), with the roofline fraction of the dominant kernel. "--impl
+reference" times the fp64 CPU oracle on the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from long_context_decode_lr_b200 import synth  # noqa: E402
+
+METRIC = "compressed-cache decode: context tokens/s per layer & % of roofline (HBM GB/s)"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(w: synth.Workload, n_sel: int):
+    """(tensor FLOPs, HBM bytes) one decode step of one layer must do at minimum.
+
+    Per attended token and KV head: the key rebuild A.B_l^h (2 r hd FLOPs) and the
+    GELU branch's first matmul (2 hd H FLOPs); W_lin and W2 are applied once per
+    query head after the softmax sums, so they do not scale with tokens. Bytes: the
+    A rows of the attended tokens (each row once), the layer's basis slice and
+    predictors per sequence, the residual rows and indices of attended tokens, the
+    block lists and the query/output.
+    """
+    e = 2
+    B, T, r, hd, H, Hkv, Hq = w.batch, w.T, w.rank, w.head_dim, w.hidden, w.n_kv_heads, w.n_q_heads
+    if n_sel:
+        # each KV head rebuilds its own n_sel blocks; A rows are moved once per distinct block
+        toks_head = min(n_sel * 64, T)
+        union = min(1.0, 1.0 - (1.0 - n_sel / w.nblk) ** Hkv)
+        a_rows = union * T
+    else:
+        toks_head = T
+        a_rows = T
+    flops = B * Hkv * toks_head * (2 * r * hd + 2 * hd * H)
+    res_frac = toks_head / T
+    bytes_ = B * (a_rows * r * e                                  # A rows
+                  + Hkv * hd * r * e                              # B_l
+                  + Hkv * (hd * hd + 2 * hd * H + H + hd) * e     # predictors
+                  + Hkv * w.k * res_frac * (hd * e + 4)           # residual rows + indices
+                  + Hkv * (w.nblk + 1) * 4                        # block pointers
+                  + Hkv * n_sel * 4                               # block lists
+                  + 2 * Hq * hd * e)                              # q and o
+    return float(flops), float(bytes_)
+
+
+class ClockSampler:
+    """Polls NVML every 20 ms: SM clock, max clock and active throttle reasons."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, n in self.REASONS.items():
+                    if bits & b and n != "gpu_idle":
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- cache
+
+def build_cache(w: synth.Workload, lr, seed_offset: int = 0):
+    """Synthetic K, V -> lr_pack_prefill on the GPU. Returns device tensors and pack timing."""
+    wr = w.replace(seed=w.seed + seed_offset)
+    mw = synth.model_weights(wr)
+    pred = synth.predictor_init(wr, mw)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    K, V, Bt = [], [], []
+    for b in range(w.batch):
+        kb, vb = synth.keys_values(wr, mw, b)
+        Bt.append(synth.key_basis_from_keys(kb, w.rank))
+        K.append(kb), V.append(vb)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
+    c = {"K": dev(np.stack(K)), "V": dev(np.stack(V)), "Bt": dev(np.stack(Bt)),
+         "W_lin": dev(pred.W_lin), "W1": dev(pred.W1), "b1": dev(pred.b1), "W2": dev(pred.W2)}
+    del K, V
+    q = synth.queries(wr, mw, 0)
+    c["q"] = [dev(synth.queries(wr, mw, l)) for l in range(w.n_layers)]
+    shape = lr.cache_shape(w.batch, w.T, w.n_layers, w.n_kv_heads, w.head_dim, w.rank, w.hidden, dt)
+    k = w.k
+    c["A"] = torch.empty((w.batch, w.T, w.rank), dtype=dt, device="cuda")
+    c["idx"] = torch.empty((w.batch, w.n_layers, w.n_kv_heads, k), dtype=torch.int32, device="cuda")
+    c["val"] = torch.empty((w.batch, w.n_layers, w.n_kv_heads, k, w.head_dim), dtype=dt, device="cuda")
+    c["ptr"] = torch.empty((w.batch, w.n_layers, w.n_kv_heads, w.nblk + 1), dtype=torch.int32, device="cuda")
+    ws = lr.workspace(lr.lr_pack_workspace_bytes(shape, k))
+    pr = lr.Predictor(c["W_lin"], c["W1"], c["b1"], c["W2"], None, True)
+    times = []
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lr.lr_pack_prefill(shape, c["K"], c["V"], c["Bt"], pr, k, c["A"], c["idx"], c["val"], c["ptr"], None, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    code = lr.lr_get_device_error(ws)
+    if code:
+        raise RuntimeError(f"pack reported device error {code}")
+    del ws
+    c.pop("K"), c.pop("V")
+    torch.cuda.empty_cache()
+    pack_ms = min(times)
+    T_tot = w.batch * w.T
+    pack_flops = T_tot * (2 * w.D * w.rank + w.n_layers * w.n_kv_heads *
+                          (2 * w.rank * w.head_dim + 2 * w.head_dim * w.hidden * 2 + 2 * w.head_dim * w.head_dim))
+    return c, shape, pr, {"ms": pack_ms, "context_tokens_per_s": T_tot / (pack_ms * 1e-3),
+                          "tflops": pack_flops / (pack_ms * 1e-3) / 1e12, "k": k}
+
+
+def clone_cache(c, lr):
+    d = {k: (v.clone() if isinstance(v, torch.Tensor) else [x.clone() for x in v]) for k, v in c.items()}
+    d["pred"] = lr.Predictor(d["W_lin"], d["W1"], d["b1"], d["W2"], None, True)
+    return d
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_lowram(args, world, rank):
+    from long_context_decode_lr_b200 import build, lowram as lr
+    if rank == 0 or world == 1:
+        build.build()
+    barrier(world)
+    lr.library()
+    w = synth.WORKLOADS[args.workload]
+    n_sel = w.n_sel
+    c0, shape, _, pack = build_cache(w, lr, seed_offset=rank)
+    per_copy = sum(t.numel() * t.element_size() for t in c0.values() if isinstance(t, torch.Tensor))
+    n_copies = max(2, math.ceil(2.2 * L2_BYTES / max(per_copy, 1)))
+    copies = [clone_cache(c0, lr) for _ in range(n_copies)]
+    del c0
+    blocks = None
+    if n_sel:
+        blocks = torch.from_numpy(synth.block_lists(w)).cuda()
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    ws = lr.workspace(lr.lr_decode_workspace_bytes(shape, w.n_q_heads, n_sel))
+    outs = [torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=dt, device="cuda") for _ in range(2)]
+    stream = torch.cuda.current_stream()
+    k = w.k
+
+    def step(i, q=None, o=None):
+        c = copies[i % n_copies]
+        layer = (i // n_copies) % w.n_layers
+        lr.lr_decode_attn(shape, layer, w.n_q_heads, c["q"][layer] if q is None else q, c["A"], c["Bt"],
+                          c["pred"], c["idx"], c["val"], c["ptr"], k, blocks, n_sel, 0.0,
+                          outs[i & 1] if o is None else o, ws, stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if lr.lr_get_device_error(ws):
+        raise RuntimeError("decode reported a device data error")
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = e0.elapsed_time(e1)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+
+    # end to end: host q (pinned) -> device, decode, output -> host, every step
+    q_host = [c["q"][l].cpu().pin_memory() for l in range(w.n_layers) for c in copies[:1]]
+    o_host = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=dt).pin_memory()
+    q_dev = torch.empty_like(copies[0]["q"][0])
+    o_dev = torch.empty_like(outs[0])
+    e_steps = max(10, min(args.steps, 200))
+    barrier(world)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(e_steps):
+        layer = (i // n_copies) % w.n_layers
+        q_dev.copy_(q_host[layer], non_blocking=True)
+        step(i, q=q_dev, o=o_dev)
+        o_host.copy_(o_dev, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1) / e_steps, world)
+
+    if rank != 0:
+        return None
+    flops, bytes_ = algorithmic_work(w, n_sel)
+    pk, pk_kind = peaks()
+    timed_s = ms_total * 1e-3
+    tpeak = pk["bf16_tflops_sustained"] if timed_s > 2.0 else pk["bf16_tflops"]
+    t_tensor = flops / (tpeak * 1e12)
+    t_hbm = bytes_ / (pk["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    s_step = ms_step * 1e-3
+    if bound == "tensor":
+        achieved, peak, unit = flops / s_step / 1e12, tpeak, "TFLOP/s"
+    else:
+        achieved, peak, unit = bytes_ / s_step / 1e9, pk["hbm_gbs"], "GB/s"
+    tokens = w.batch * w.T * world
+    value = tokens / s_step
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "description": w.description, "batch_per_gpu": w.batch,
+                   "context": w.T, "mode": "selective" if n_sel else "full", "n_sel": n_sel,
+                   "residual_pct": w.res_pct, "step": "one lr_decode_attn call (one layer)",
+                   "l2": f"inputs rotate over {n_copies} device copies of the cache "
+                         f"({n_copies * per_copy / 2**20:.0f} MB > L2)",
+                   "parallelism": f"dp{world}" if world > 1 else "single"},
+        "us_per_layer": ms_step * 1e3, "model_32_layers_ms": ms_step * 32,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None,
+                     "kernel": "lr_decode_attn (split kernel + combine; event time covers both)",
+                     "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
+                     "peak_source": f"{pk_kind} ({'sustained' if tpeak == pk.get('bf16_tflops_sustained') else 'burst'} bf16)"},
+        "roofline_pct": 100.0 * max(t_tensor, t_hbm) / s_step,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
+                "d2h_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "pack": pack,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_seconds)
+    return out
+
+
+def _oracle_inputs(w: synth.Workload):
+    """fp64 inputs for the oracle: a compressed cache drawn directly at the workload's size."""
+    mw = synth.model_weights(w)
+    pred = synth.predictor_init(w, mw, batch=1)
+    c = synth.decode_cache(w, mw, batch=1)
+    f = lambda a: synth.to_storage(a, w.dtype)[1]
+    q = f(synth.queries(w, mw, 0, batch=1))
+    return dict(A=f(c.A[0]), Bt=f(c.Bt[0]), W_lin=f(pred.W_lin[0]), W1=f(pred.W1[0]), b1=f(pred.b1[0]),
+                W2=f(pred.W2[0]), idx=c.res_idx[0].astype(np.int64), val=f(c.res_val[0]), q=q[0])
+
+
+def _oracle_one_head(w, d, h, blocks):
+    from oracle import lowram_oracle as orc
+    G = w.q_per_kv
+    sub = lambda a: a[:, h:h + 1]
+    Bt_h = d["Bt"][(0 * w.n_kv_heads + h) * w.head_dim:][: w.head_dim]
+    # one KV head of layer 0 through the oracle, as a one-head problem
+    return orc.decode_sequence(d["q"][h * G:(h + 1) * G], d["A"], Bt_h, sub(d["W_lin"]), sub(d["W1"]),
+                               sub(d["b1"]), sub(d["W2"]), None, 0, sub(d["idx"]), sub(d["val"]),
+                               None if blocks is None else blocks[h:h + 1], orc.default_scale(w.head_dim, 0),
+                               1, w.head_dim)
+
+
+def cpu_baseline(w: synth.Workload, budget_s: float = 15.0):
+    """Time the oracle on the host: one KV head (G query heads) of one layer per sample."""
+    d = _oracle_inputs(w)
+    blocks = synth.block_lists(w, batch=1)[0] if w.n_sel else None
+    times = []
+    t_start = time.perf_counter()
+    h = 0
+    while True:
+        t0 = time.perf_counter()
+        _oracle_one_head(w, d, h % w.n_kv_heads, blocks)
+        times.append(time.perf_counter() - t0)
+        h += 1
+        if time.perf_counter() - t_start > budget_s or h >= 64:
+            break
+    t_head = statistics.median(times)
+    t_layer = t_head * w.n_kv_heads * w.batch
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": w.batch * w.T / t_layer, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"fp64 oracle decode of one KV head ({w.q_per_kv} query heads) over all {w.T} tokens "
+                      f"of one sequence, {len(times)} samples (median {t_head:.3f} s); scaled x{w.n_kv_heads} "
+                      f"heads x{w.batch} sequences to one layer step"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = synth.WORKLOADS[args.workload]
+    d = _oracle_inputs(w)
+    blocks = synth.block_lists(w, batch=1)[0] if w.n_sel else None
+    for i in range(args.warmup):
+        _oracle_one_head(w, d, i % w.n_kv_heads, blocks)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        _oracle_one_head(w, d, i % w.n_kv_heads, blocks)
+    dt = (time.perf_counter() - t0) / args.steps
+    t_layer = dt * w.n_kv_heads * w.batch
+    value = w.batch * w.T / t_layer
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    sample = (f"each step: fp64 oracle decode of one KV head ({w.q_per_kv} query heads) over all {w.T} tokens; "
+              f"step time x{w.n_kv_heads} heads x{w.batch} sequences = one layer")
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_layer * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "description": w.description, "context": w.T,
+                       "mode": "selective" if w.n_sel else "full"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["lowram", "reference"], default="lowram")
+    ap.add_argument("--workload", default="mistral_group_32k", choices=synth.names())
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, _ = dist_setup(args.gpus)
+    try:
+        out = run_lowram(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,210 @@
+/*
+ * lowram.h -- C ABI of the LowRAM compressed-KV-cache path for NVIDIA B200 (sm_100a).
+ *
+ * The method (LowRAM: low-rank keys and amortised values):
+ *   - "LowRAM" project page, Figure 3: the keys of a group of adjacent layers are
+ *     stored as one shared per-token factor A and a smaller per-layer factor, so
+ *     the keys of layer l are A . B_l.
+ *   - "Predicting the value cache from keys" explainer, paragraphs 2-4: values are
+ *     not stored; a small per-KV-head network rebuilds them from the keys (a
+ *     pseudoinverse-initialised linear map plus a GELU branch), and exact residual
+ *     corrections are kept for the tokens it predicts worst, ranked by error.
+ *   - arXiv 2611.07025 abstract: at each decode step only a selected subset of the
+ *     cached pairs needs to be rebuilt (selective reconstruction).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE memory owned by the caller. The library never
+ *     allocates device memory, never frees caller memory and keeps no state between
+ *     calls; scratch space is the caller's workspace (`ws`, `ws_bytes`).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) in stream order. No entry point synchronises the host except
+ *     lr_get_device_error.
+ *   - Floating tensors all use the storage type `dtype` of the cache shape
+ *     (LR_BF16 or LR_F32); arithmetic is fp32 with fp32 accumulation.
+ *     Index tensors are int32. Every tensor is dense, row-major, with the
+ *     dimensions listed (leftmost slowest).
+ *   - Data pointers must be 16-byte aligned; the workspace 256-byte aligned.
+ *   - Host-side checks (null pointers, shapes, alignment, workspace size) run
+ *     before any launch and return a status without touching device memory.
+ *     LR_ERR_CUDA means a launch failed (cudaGetLastError). Device-side data
+ *     checks (out-of-range or unsorted indices) skip the offending entry and set
+ *     bits in an error word inside the workspace; read it with
+ *     lr_get_device_error. No kernel traps, asserts or spins.
+ *   - The last failing host-side check's message is available, per thread, from
+ *     lr_last_error().
+ *
+ * Notation: B batch (sequences), T context tokens, L_g layers per group,
+ * Hkv KV heads, G = Hq / Hkv query heads per KV head (query head hq reads KV
+ * head hq / G), hd head_dim, D = L_g * Hkv * hd, r key rank, H predictor
+ * hidden width, k residual rows per (sequence, layer, KV head),
+ * nblk = ceil(T / 64) key blocks of 64 tokens.
+ */
+#ifndef LOWRAM_H
+#define LOWRAM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LR_ABI_VERSION 1
+#define LR_BLOCK_TOKENS 64
+
+typedef void* lr_stream_t; /* cudaStream_t */
+
+typedef enum lr_status {
+  LR_OK = 0,
+  LR_ERR_INVALID_ARG = 1,  /* a null pointer, bad size, bad alignment or out-of-range argument */
+  LR_ERR_UNSUPPORTED = 2,  /* a valid shape this build does not implement */
+  LR_ERR_WORKSPACE = 3,    /* ws_bytes below the size the matching *_workspace_bytes returns */
+  LR_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
+  LR_ERR_DEVICE_CHECK = 5  /* lr_get_device_error found a nonzero device error word */
+} lr_status;
+
+typedef enum lr_dtype { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
+
+/* Bits of the device error word (OR-ed over one call). */
+#define LR_DEVERR_BLOCK_RANGE 1 /* a selected block id outside [0, nblk): entry skipped */
+#define LR_DEVERR_BLOCK_ORDER 2 /* selected block ids not strictly ascending: entry skipped */
+#define LR_DEVERR_RES_RANGE 4   /* a residual index outside its block or [0, T): entry skipped */
+#define LR_DEVERR_RES_ORDER 8   /* residual indices not strictly ascending */
+#define LR_DEVERR_PTR 16        /* a residual block pointer out of [0, k] or decreasing */
+
+typedef struct lr_cache_shape {
+  int32_t batch;      /* B >= 0 */
+  int32_t T;          /* context tokens per sequence, >= 0 */
+  int32_t n_layers;   /* L_g >= 1: layers sharing one key factor A */
+  int32_t n_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;   /* hd: multiple of 8, <= 256 */
+  int32_t rank;       /* r: multiple of 8, >= 8 */
+  int32_t hidden;     /* H: predictor hidden width, multiple of 8, <= 1024 */
+  lr_dtype dtype;     /* storage type of every floating tensor */
+} lr_cache_shape;
+
+/*
+ * Value predictor f_theta of every (layer, KV head) of the group ("Predicting
+ * the value cache from keys", paragraphs 2-3):
+ *     v_hat = k W_lin^T + GELU(k W1^T + b1) W2^T + b2,   GELU(x) = x Phi(x) (erf form),
+ * where k is the reconstructed key of one token and one KV head. Weights are in
+ * nn.Linear layout (out x in). With per_sequence = 1 every array has a leading
+ * batch dimension [B, ...]; with 0 one predictor serves all sequences.
+ *     W_lin [(B,) L_g, Hkv, hd, hd]     W1 [(B,) L_g, Hkv, H, hd]     b1 [(B,) L_g, Hkv, H]
+ *     W2    [(B,) L_g, Hkv, hd, H]      b2 [(B,) L_g, Hkv, hd] or NULL (= zero)
+ */
+typedef struct lr_predictor {
+  const void* W_lin;
+  const void* W1;
+  const void* b1;
+  const void* W2;
+  const void* b2;
+  int32_t per_sequence;
+} lr_predictor;
+
+/* ------------------------------------------------------------------ prefill packer */
+
+/* Workspace bytes lr_pack_prefill needs for this shape and residual count. */
+size_t lr_pack_workspace_bytes(const lr_cache_shape* shape, int32_t k);
+
+/*
+ * lr_pack_prefill -- build the compressed cache of one layer group.
+ *
+ * Steps (project page Figure 3; explainer paragraphs 2-4):
+ *   1. A = round(K_group . Bt): project every token's group keys onto the shared
+ *      factor (Bt has orthonormal columns: the truncated-SVD basis B transposed).
+ *   2. For each layer l and KV head h: k~_t = A[t] . B_l^h, where B_l^h is rows
+ *      (l*Hkv + h)*hd .. +hd of Bt;
+ *   3. v_hat_t = f_theta(k~_t) with the (l, h) predictor;
+ *   4. e_t = sum_j (v_t[j] - v_hat_t[j])^2 (fp32);
+ *   5. the k tokens of largest e_t, ties to the lower token index, ascending;
+ *   6. res_val = round(v - v_hat) at those tokens, and the block pointers
+ *      res_blk_ptr[j] = #{i : res_idx[i] < 64 j}, j = 0 .. nblk.
+ *   round() is round-to-nearest-even to the storage type.
+ *
+ * Inputs:  K_group [B, T, D]; V [B, L_g, T, Hkv, hd]; Bt [B, D, r];
+ *          predictor as above; 0 <= k <= T.
+ * Outputs: A [B, T, r]; res_idx [B, L_g, Hkv, k] int32; res_val [B, L_g, Hkv, k, hd];
+ *          res_blk_ptr [B, L_g, Hkv, nblk + 1] int32 or NULL;
+ *          err_out [B, L_g, Hkv, T] fp32 or NULL (the e_t of step 4).
+ * res_idx / res_val may be NULL when k == 0.
+ */
+lr_status lr_pack_prefill(const lr_cache_shape* shape, const void* K_group, const void* V,
+                          const void* Bt, const lr_predictor* predictor, int32_t k, void* A,
+                          int32_t* res_idx, void* res_val, int32_t* res_blk_ptr, float* err_out,
+                          void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/* ------------------------------------------------------------------ decode attention */
+
+/* Workspace bytes lr_decode_attn needs (n_sel = 0 for full reconstruction). The
+ * answer depends on the current device's SM count; query it on the device that runs
+ * the call. */
+size_t lr_decode_workspace_bytes(const lr_cache_shape* shape, int32_t n_q_heads, int32_t n_sel);
+
+/*
+ * lr_decode_attn -- one decode step of one layer over the compressed cache.
+ *
+ * For each sequence b and query head hq (KV head h = hq / G):
+ *   S    = all tokens [0, T) when block_list is NULL, else the union of the 64-token
+ *          blocks block_list[b, h, 0 .. n_sel) (selective reconstruction, arXiv
+ *          abstract); the last block is clipped at T;
+ *   k~_t = A[b, t] . B_l^h                         (project page, Figure 3)
+ *   v_t  = f_theta(k~_t) + res_val[i]  if t = res_idx[b, l, h, i], else f_theta(k~_t)
+ *                                                  (explainer, paragraph 2)
+ *   o[b, hq] = sum_{t in S} softmax_t(scale * q[b, hq] . k~_t) v_t
+ * An empty S gives o = 0. scale <= 0 selects 1/sqrt(hd).
+ *
+ * Inputs:  q [B, Hq, hd]; A [B, T, r]; Bt [B, D, r]; predictor of the group;
+ *          res_idx [B, L_g, Hkv, k] ascending per row; res_val [B, L_g, Hkv, k, hd];
+ *          res_blk_ptr [B, L_g, Hkv, nblk + 1] or NULL (then the kernel searches res_idx);
+ *          block_list [B, Hkv, n_sel] strictly ascending block ids, or NULL = all tokens;
+ *          0 <= layer < L_g; n_q_heads a multiple of Hkv; 0 <= n_sel <= nblk.
+ * Output:  o [B, Hq, hd].
+ */
+lr_status lr_decode_attn(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
+                         const void* q, const void* A, const void* Bt,
+                         const lr_predictor* predictor, const int32_t* res_idx,
+                         const void* res_val, const int32_t* res_blk_ptr, int32_t k,
+                         const int32_t* block_list, int32_t n_sel, float scale, void* o,
+                         void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/* ------------------------------------------------------------------ single steps */
+
+/* Workspace bytes lr_topk_tokens needs. */
+size_t lr_topk_workspace_bytes(int32_t n_segments, int32_t T, int32_t k);
+
+/*
+ * lr_topk_tokens -- step 5 of the packer on its own (explainer, paragraph 4:
+ * residuals go to the tokens ranked worst by error).
+ * err [n_segments, T] fp32 -> idx_out [n_segments, k] int32: per segment the k
+ * tokens of largest error, ties to the lower index, in ascending index order.
+ * Errors compare as IEEE values (-0 == +0); NaN ranks below every number.
+ * The result is unique, so it is bit-exact by definition.
+ */
+lr_status lr_topk_tokens(const float* err, int32_t n_segments, int32_t T, int32_t k,
+                         int32_t* idx_out, void* ws, size_t ws_bytes, lr_stream_t stream);
+
+/*
+ * lr_residual_block_ptr -- the residual block pointers of step 6 on their own.
+ * idx [n_segments, k] ascending -> ptr_out [n_segments, nblk + 1] with
+ * ptr_out[s, j] = #{i : idx[s, i] < 64 j}. Needs no workspace.
+ */
+lr_status lr_residual_block_ptr(const int32_t* idx, int32_t n_segments, int32_t k, int32_t T,
+                                int32_t* ptr_out, lr_stream_t stream);
+
+/* ------------------------------------------------------------------ errors, version */
+
+/* Copies the device error word of the last call that used `ws` into *code and
+ * synchronises `stream`. Returns LR_OK when the word is 0, LR_ERR_DEVICE_CHECK when it
+ * is not, LR_ERR_CUDA when the copy fails. Every call that takes a workspace clears
+ * the word when it starts. */
+lr_status lr_get_device_error(const void* ws, lr_stream_t stream, int32_t* code);
+
+const char* lr_status_string(lr_status status);
+const char* lr_last_error(void);
+int32_t lr_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LOWRAM_H */

@@ -1,0 +1,255 @@
+// Host side of the C ABI declared in include/lowram.h: argument checks, workspace
+// planning and kernel launches. Nothing here allocates device memory or keeps
+// state between calls; the only per-thread state is the last error message.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "lowram.h"
+#include "lr_common.cuh"
+#include "lr_launch.h"
+#include "lr_plan.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+lr_status fail(lr_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lr_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(LR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+#define CHECK_PTR(p, name)                                                          \
+  do {                                                                              \
+    if (!(p)) return fail(LR_ERR_INVALID_ARG, "%s is NULL", name);                  \
+    if (!aligned((p), 16)) return fail(LR_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+#define CHECK_OPT_PTR(p, name)                                                      \
+  do {                                                                              \
+    if ((p) && !aligned((p), 16)) return fail(LR_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+lr_status check_shape(const lr_cache_shape* s) {
+  if (!s) return fail(LR_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 0 || s->T < 0) return fail(LR_ERR_INVALID_ARG, "batch and T must be >= 0");
+  if (s->n_layers < 1 || s->n_kv_heads < 1) return fail(LR_ERR_INVALID_ARG, "n_layers and n_kv_heads must be >= 1");
+  if (s->head_dim < 1 || s->rank < 1 || s->hidden < 1) return fail(LR_ERR_INVALID_ARG, "head_dim, rank and hidden must be >= 1");
+  if (s->dtype != LR_F32 && s->dtype != LR_BF16) return fail(LR_ERR_INVALID_ARG, "unknown dtype %d", (int)s->dtype);
+  if (s->head_dim % 8 || s->head_dim > 256) return fail(LR_ERR_UNSUPPORTED, "head_dim must be a multiple of 8 and <= 256");
+  if (s->rank % 8) return fail(LR_ERR_UNSUPPORTED, "rank must be a multiple of 8");
+  if (s->hidden % 8 || s->hidden > 512) return fail(LR_ERR_UNSUPPORTED, "hidden must be a multiple of 8 and <= 512");
+  const long long D = (long long)s->n_layers * s->n_kv_heads * s->head_dim;
+  if (D > (1 << 20)) return fail(LR_ERR_UNSUPPORTED, "layer-group key width too large");
+  return LR_OK;
+}
+
+lr_status check_predictor(const lr_predictor* p) {
+  if (!p) return fail(LR_ERR_INVALID_ARG, "predictor is NULL");
+  CHECK_PTR(p->W_lin, "predictor.W_lin");
+  CHECK_PTR(p->W1, "predictor.W1");
+  CHECK_PTR(p->b1, "predictor.b1");
+  CHECK_PTR(p->W2, "predictor.W2");
+  CHECK_OPT_PTR(p->b2, "predictor.b2");
+  if (p->per_sequence != 0 && p->per_sequence != 1) return fail(LR_ERR_INVALID_ARG, "predictor.per_sequence must be 0 or 1");
+  return LR_OK;
+}
+
+lr_status check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(LR_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(ws, 256)) return fail(LR_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  if (ws_bytes < need) return fail(LR_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, need);
+  return LR_OK;
+}
+
+int current_sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  return n;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lr_last_error(void) { return g_msg; }
+
+int32_t lr_abi_version(void) { return LR_ABI_VERSION; }
+
+const char* lr_status_string(lr_status s) {
+  switch (s) {
+    case LR_OK: return "ok";
+    case LR_ERR_INVALID_ARG: return "invalid argument";
+    case LR_ERR_UNSUPPORTED: return "unsupported shape";
+    case LR_ERR_WORKSPACE: return "workspace too small";
+    case LR_ERR_CUDA: return "CUDA error";
+    case LR_ERR_DEVICE_CHECK: return "device-side data check failed";
+  }
+  return "unknown status";
+}
+
+lr_status lr_get_device_error(const void* ws, lr_stream_t stream, int32_t* code) {
+  if (!ws || !code) return fail(LR_ERR_INVALID_ARG, "ws and code must not be NULL");
+  int32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+  *code = v;
+  return v ? LR_ERR_DEVICE_CHECK : LR_OK;
+}
+
+// ------------------------------------------------------------------ decode
+
+size_t lr_decode_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads, int32_t n_sel) {
+  if (check_shape(s) != LR_OK || n_q_heads < 1) return 0;
+  return lr::plan_decode(*s, n_q_heads, n_sel, current_sm_count()).ws_bytes;
+}
+
+lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
+                         const void* A, const void* Bt, const lr_predictor* pred,
+                         const int32_t* res_idx, const void* res_val, const int32_t* res_blk_ptr,
+                         int32_t k, const int32_t* block_list, int32_t n_sel, float scale, void* o,
+                         void* ws, size_t ws_bytes, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (layer < 0 || layer >= s->n_layers) return fail(LR_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, s->n_layers);
+  if (n_q_heads < 1 || n_q_heads % s->n_kv_heads) return fail(LR_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (n_q_heads / s->n_kv_heads > 8) return fail(LR_ERR_UNSUPPORTED, "more than 8 query heads per KV head");
+  const int nblk = lr::ceil_div(s->T, LR_BLOCK_TOKENS);
+  if (k < 0 || k > s->T) return fail(LR_ERR_INVALID_ARG, "k=%d outside [0, T]", k);
+  if (block_list && (n_sel < 0 || n_sel > nblk)) return fail(LR_ERR_INVALID_ARG, "n_sel=%d outside [0, nblk=%d]", n_sel, nblk);
+  if (!block_list) n_sel = 0;
+  if ((st = check_predictor(pred)) != LR_OK) return st;
+  CHECK_PTR(q, "q");
+  CHECK_PTR(A, "A");
+  CHECK_PTR(Bt, "Bt");
+  CHECK_PTR(o, "o");
+  if (k > 0) {
+    CHECK_PTR(res_idx, "res_idx");
+    CHECK_PTR(res_val, "res_val");
+  }
+  CHECK_OPT_PTR(res_blk_ptr, "res_blk_ptr");
+  CHECK_OPT_PTR(block_list, "block_list");
+  const lr::DecodePlan plan = lr::plan_decode(*s, n_q_heads, n_sel, current_sm_count());
+  if ((st = check_ws(ws, ws_bytes, plan.ws_bytes)) != LR_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  if (s->batch == 0) return LR_OK;
+
+  lr::DecodeArgs a{};
+  a.B = s->batch; a.T = s->T; a.L = s->n_layers; a.Hkv = s->n_kv_heads; a.G = n_q_heads / s->n_kv_heads;
+  a.hd = s->head_dim; a.r = s->rank; a.H = s->hidden;
+  a.layer = layer; a.k = k; a.n_sel = n_sel; a.nblk = nblk;
+  a.pred_per_seq = pred->per_sequence;
+  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)s->head_dim);
+  a.q = q; a.A = A; a.Bt = Bt;
+  a.W_lin = pred->W_lin; a.W1 = pred->W1; a.b1 = pred->b1; a.W2 = pred->W2; a.b2 = pred->b2;
+  a.res_idx = k ? res_idx : nullptr; a.res_val = k ? res_val : nullptr;
+  a.res_ptr = k ? res_blk_ptr : nullptr;
+  a.blocks = block_list;
+  a.o = o;
+  a.err = (int*)ws;
+  a.partials = (float*)((char*)ws + plan.part_off);
+  a.n_split = plan.n_split;
+  a.part_stride = plan.part_stride;
+  if ((e = lr::launch_decode(a, plan, s->dtype, cs)) != cudaSuccess) return cuda_fail(e, "decode launch");
+  return LR_OK;
+}
+
+// ------------------------------------------------------------------ pack
+
+size_t lr_pack_workspace_bytes(const lr_cache_shape* s, int32_t k) {
+  if (check_shape(s) != LR_OK || k < 0) return 0;
+  return lr::plan_pack(*s, k).ws_bytes;
+}
+
+lr_status lr_pack_prefill(const lr_cache_shape* s, const void* K_group, const void* V, const void* Bt,
+                          const lr_predictor* pred, int32_t k, void* A, int32_t* res_idx,
+                          void* res_val, int32_t* res_blk_ptr, float* err_out, void* ws,
+                          size_t ws_bytes, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (k < 0 || k > s->T) return fail(LR_ERR_INVALID_ARG, "k=%d outside [0, T]", k);
+  if ((st = check_predictor(pred)) != LR_OK) return st;
+  CHECK_PTR(K_group, "K_group");
+  CHECK_PTR(V, "V");
+  CHECK_PTR(Bt, "Bt");
+  CHECK_PTR(A, "A");
+  if (k > 0) {
+    CHECK_PTR(res_idx, "res_idx");
+    CHECK_PTR(res_val, "res_val");
+  }
+  CHECK_OPT_PTR(res_blk_ptr, "res_blk_ptr");
+  CHECK_OPT_PTR(err_out, "err_out");
+  const lr::PackPlan plan = lr::plan_pack(*s, k);
+  if ((st = check_ws(ws, ws_bytes, plan.ws_bytes)) != LR_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  if (s->batch == 0) return LR_OK;
+
+  lr::PackArgs a{};
+  a.B = s->batch; a.T = s->T; a.L = s->n_layers; a.Hkv = s->n_kv_heads; a.hd = s->head_dim;
+  a.r = s->rank; a.H = s->hidden; a.D = s->n_layers * s->n_kv_heads * s->head_dim; a.k = k;
+  a.nblk = lr::ceil_div(s->T, LR_BLOCK_TOKENS);
+  a.pred_per_seq = pred->per_sequence;
+  a.K = K_group; a.V = V; a.Bt = Bt;
+  a.W_lin = pred->W_lin; a.W1 = pred->W1; a.b1 = pred->b1; a.W2 = pred->W2; a.b2 = pred->b2;
+  a.A = A;
+  a.err = err_out ? err_out : (float*)((char*)ws + plan.err_off);
+  a.diff = (char*)ws + plan.diff_off;
+  a.res_idx = res_idx; a.res_val = res_val; a.res_ptr = res_blk_ptr;
+  a.errword = (int*)ws;
+  if ((e = lr::launch_pack(a, plan, s->dtype, cs)) != cudaSuccess) return cuda_fail(e, "pack launch");
+  return LR_OK;
+}
+
+// ------------------------------------------------------------------ single steps
+
+size_t lr_topk_workspace_bytes(int32_t n_segments, int32_t T, int32_t k) {
+  (void)n_segments; (void)T; (void)k;
+  return 256;
+}
+
+lr_status lr_topk_tokens(const float* err, int32_t n_segments, int32_t T, int32_t k, int32_t* idx_out,
+                         void* ws, size_t ws_bytes, lr_stream_t stream) {
+  if (n_segments < 0 || T < 0) return fail(LR_ERR_INVALID_ARG, "n_segments and T must be >= 0");
+  if (k < 0 || k > T) return fail(LR_ERR_INVALID_ARG, "k=%d outside [0, T]", k);
+  lr_status st = check_ws(ws, ws_bytes, 256);
+  if (st != LR_OK) return st;
+  if (n_segments > 0 && k > 0) {
+    CHECK_PTR(err, "err");
+    CHECK_PTR(idx_out, "idx_out");
+  }
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, cs);
+  if (e == cudaSuccess) e = lr::launch_topk(err, n_segments, T, k, idx_out, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "top-k launch");
+  return LR_OK;
+}
+
+lr_status lr_residual_block_ptr(const int32_t* idx, int32_t n_segments, int32_t k, int32_t T,
+                                int32_t* ptr_out, lr_stream_t stream) {
+  if (n_segments < 0 || T < 0) return fail(LR_ERR_INVALID_ARG, "n_segments and T must be >= 0");
+  if (k < 0 || k > T) return fail(LR_ERR_INVALID_ARG, "k=%d outside [0, T]", k);
+  if (n_segments == 0) return LR_OK;
+  if (k > 0) CHECK_PTR(idx, "idx");
+  CHECK_PTR(ptr_out, "ptr_out");
+  cudaError_t e = lr::launch_block_ptr(idx, n_segments, k, T, ptr_out, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block pointer launch");
+  return LR_OK;
+}
+
+}  // extern "C"

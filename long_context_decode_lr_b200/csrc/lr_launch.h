@@ -1,0 +1,29 @@
+// Host-side launch functions of the LowRAM kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "lowram.h"
+
+namespace lr {
+
+struct DecodeArgs;
+struct PackArgs;
+
+// General CUDA-core decode path (any supported shape, fp32 or bf16 storage).
+size_t decode_general_smem_bytes(int hd, int H, int G);
+size_t decode_combine_smem_bytes(int hd, int H, int n_split);
+cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t st);
+cudaError_t launch_decode_combine(const DecodeArgs& a, lr_dtype dt, cudaStream_t st);
+
+// Packer steps.
+cudaError_t launch_pack_project_general(const PackArgs& a, lr_dtype dt, cudaStream_t st);
+cudaError_t launch_pack_predict_general(const PackArgs& a, lr_dtype dt, cudaStream_t st);
+cudaError_t launch_pack_gather(const PackArgs& a, lr_dtype dt, cudaStream_t st);
+
+// Top-k token selection (radix select) and residual block pointers.
+cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st);
+cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_out, cudaStream_t st);
+
+}  // namespace lr

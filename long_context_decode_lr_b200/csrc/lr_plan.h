@@ -1,0 +1,38 @@
+// Workspace plans and kernel dispatch of the decode and pack calls (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "lowram.h"
+
+namespace lr {
+
+struct DecodeArgs;
+struct PackArgs;
+
+enum class DecodePath { General = 0, Tensor = 1 };
+
+struct DecodePlan {
+  DecodePath path;
+  int n_split;       // token splits per (sequence, KV head) (general) or per sequence (tensor)
+  int part_stride;   // floats per split partial
+  size_t part_off;   // byte offset of the partials in the workspace
+  size_t sched_off;  // byte offset of the tensor path's block schedule
+  size_t ws_bytes;   // total workspace
+};
+
+struct PackPlan {
+  bool tensor;       // tensor-core projection / prediction kernels
+  size_t err_off;    // fp32 errors when the caller passes no err_out
+  size_t diff_off;   // round(v - v_hat) for every token
+  size_t ws_bytes;
+};
+
+DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);
+PackPlan plan_pack(const lr_cache_shape& s, int k);
+
+cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype dt, cudaStream_t st);
+cudaError_t launch_pack(const PackArgs& a, const PackPlan& plan, lr_dtype dt, cudaStream_t st);
+
+}  // namespace lr

@@ -1,0 +1,157 @@
+// Residual token selection ("Predicting the value cache from keys", paragraph 4:
+// exact corrections go to the tokens the predictor reconstructs worst).
+//
+// Per segment (one (sequence, layer, KV head)) the k tokens of largest error are
+// chosen, ties to the lower token index, and written in ascending index order.
+// Errors are mapped to order-preserving 32-bit keys; an MSB-first radix select
+// (four 8-bit passes with warp-aggregated shared-memory histograms) finds the key
+// K* of the k-th largest error and how many tokens tie at K*; one ordered
+// compaction pass then emits every token above K* plus the lowest-index ties.
+// Every (key, index) pair is distinct, so the result is unique and the step is
+// exact integer work.
+#include "lr_common.cuh"
+#include "lr_launch.h"
+
+namespace lr {
+namespace {
+
+constexpr int TK_THREADS = 1024;
+constexpr int TK_WARPS = TK_THREADS / 32;
+
+// IEEE order as unsigned order; -0 maps with +0, NaN below every number.
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive prefix of one flag per thread over the block; returns the block total.
+__device__ __forceinline__ int block_exclusive_scan(bool flag, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(bal);
+  __syncthreads();
+  int before = 0, sum = 0;
+  for (int w = 0; w < TK_WARPS; ++w) {
+    const int c = warp_tot[w];
+    if (w < warp) before += c;
+    sum += c;
+  }
+  total = sum;
+  __syncthreads();
+  return before + in_warp;
+}
+
+__global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ err, int T, int k,
+                                                         int* __restrict__ out_all) {
+  __shared__ int whist[TK_WARPS][256];
+  __shared__ int hist[256];
+  __shared__ int sh_digit, sh_kr;
+  __shared__ int warp_tot[TK_WARPS];
+  const int seg = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float* e = err + (size_t)seg * T;
+  int* out = out_all + (size_t)seg * k;
+  if (k == 0) return;
+  if (k == T) {
+    for (int t = tid; t < T; t += TK_THREADS) out[t] = t;
+    return;
+  }
+  uint32_t prefix = 0, mask = 0;
+  int kr = k;  // rank still to locate among keys that match the prefix
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < TK_WARPS * 256; i += TK_THREADS) (&whist[0][0])[i] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < T; t0 += TK_THREADS) {
+      const int t = t0 + tid;
+      bool act = false;
+      int digit = 0;
+      if (t < T) {
+        const uint32_t key = order_key(e[t]);
+        act = (key & mask) == prefix;
+        digit = (key >> shift) & 255;
+      }
+      const unsigned actmask = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const unsigned same = __match_any_sync(actmask, digit);
+        if ((__ffs(same) - 1) == lane) atomicAdd(&whist[warp][digit], __popc(same));
+      }
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int s = 0;
+      for (int w = 0; w < TK_WARPS; ++w) s += whist[w][tid];
+      hist[tid] = s;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, d = 255;
+      for (; d > 0; --d) {
+        if (cum + hist[d] >= kr) break;
+        cum += hist[d];
+      }
+      sh_digit = d;
+      sh_kr = kr - cum;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)sh_digit << shift;
+    mask |= 255u << shift;
+    kr = sh_kr;
+    __syncthreads();
+  }
+  // prefix is the key of the k-th largest error; kr ties at that key are taken.
+  const uint32_t kstar = prefix;
+  const int n_tie = kr;
+  int ties_before = 0, taken_before = 0;
+  for (int t0 = 0; t0 < T; t0 += TK_THREADS) {
+    const int t = t0 + tid;
+    uint32_t key = 0;
+    const bool valid = t < T;
+    if (valid) key = order_key(e[t]);
+    const bool is_eq = valid && key == kstar;
+    int eq_total;
+    const int eq_rank = ties_before + block_exclusive_scan(is_eq, warp_tot, eq_total);
+    const bool take = valid && (key > kstar || (is_eq && eq_rank < n_tie));
+    int take_total;
+    const int pos = taken_before + block_exclusive_scan(take, warp_tot, take_total);
+    if (take) out[pos] = t;
+    ties_before += eq_total;
+    taken_before += take_total;
+    if (taken_before >= k) break;
+  }
+}
+
+__global__ void block_ptr_kernel(const int* __restrict__ idx, int n_seg, int k, int T, int nblk,
+                                 int* __restrict__ ptr) {
+  const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (x >= (long long)n_seg * (nblk + 1)) return;
+  const int seg = (int)(x / (nblk + 1)), j = (int)(x % (nblk + 1));
+  const int* a = idx + (size_t)seg * k;
+  const int key = j * kBlock;
+  int lo = 0, hi = k;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  ptr[x] = lo;
+}
+
+}  // namespace
+
+cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st) {
+  if (n_seg == 0 || k == 0) return cudaSuccess;
+  topk_kernel<<<n_seg, TK_THREADS, 0, st>>>(err, T, k, idx_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_out, cudaStream_t st) {
+  const int nblk = ceil_div(T, kBlock);
+  const long long n = (long long)n_seg * (nblk + 1);
+  if (n == 0) return cudaSuccess;
+  block_ptr_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(idx, n_seg, k, T, nblk, ptr_out);
+  return cudaGetLastError();
+}
+
+}  // namespace lr

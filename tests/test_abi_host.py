@@ -1,0 +1,115 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before touching any device memory (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_decode_lr_b200 import build as lrbuild
+from long_context_decode_lr_b200 import lowram as lr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lrbuild.build()
+    return lr.library()
+
+
+def declared_functions():
+    names = set()
+    for hdr in os.listdir(os.path.join(ROOT, "include")):
+        if hdr.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", hdr)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(lr_[a-z0-9_]+)\s*\(", txt))
+    return sorted(names)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "lr_decode_attn" in names and "lr_pack_prefill" in names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_strings(lib):
+    assert lib.lr_abi_version() == 1
+    assert lib.lr_status_string(lr.LR_ERR_WORKSPACE) == b"workspace too small"
+
+
+FAKE = 0x10000  # a 256-byte-aligned address that is never dereferenced
+
+
+def _shape(**kw):
+    d = dict(batch=1, T=1000, n_layers=2, n_kv_heads=2, head_dim=128, rank=128, hidden=256, dtype=lr.LR_BF16)
+    d.update(kw)
+    return lr.lr_cache_shape(*[d[f] for f, _ in lr.lr_cache_shape._fields_])
+
+
+def _pred(**kw):
+    d = dict(W_lin=FAKE, W1=FAKE, b1=FAKE, W2=FAKE, b2=None, per_sequence=1)
+    d.update(kw)
+    return lr.lr_predictor(*[d[f] for f, _ in lr.lr_predictor._fields_])
+
+
+def _decode(lib, shape=None, layer=0, hq=8, q=FAKE, res_idx=FAKE, res_val=FAKE, k=10, blocks=None, n_sel=0,
+            pred=None, ws=FAKE, ws_bytes=1 << 40, o=FAKE):
+    shape = _shape() if shape is None else shape
+    pred = _pred() if pred is None else pred
+    return lib.lr_decode_attn(ctypes.byref(shape), layer, hq, q, FAKE, FAKE, ctypes.byref(pred), res_idx,
+                              res_val, None, k, blocks, n_sel, 0.0, o, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layer=2), lr.LR_ERR_INVALID_ARG),
+    (dict(layer=-1), lr.LR_ERR_INVALID_ARG),
+    (dict(hq=7), lr.LR_ERR_INVALID_ARG),
+    (dict(hq=2 * 16), lr.LR_ERR_UNSUPPORTED),
+    (dict(k=1001), lr.LR_ERR_INVALID_ARG),
+    (dict(k=-1), lr.LR_ERR_INVALID_ARG),
+    (dict(q=None), lr.LR_ERR_INVALID_ARG),
+    (dict(q=FAKE + 4), lr.LR_ERR_INVALID_ARG),
+    (dict(res_idx=None), lr.LR_ERR_INVALID_ARG),
+    (dict(o=None), lr.LR_ERR_INVALID_ARG),
+    (dict(blocks=FAKE, n_sel=17), lr.LR_ERR_INVALID_ARG),
+    (dict(ws=None), lr.LR_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 16), lr.LR_ERR_INVALID_ARG),
+    (dict(ws_bytes=100), lr.LR_ERR_WORKSPACE),
+    (dict(shape=_shape(head_dim=100)), lr.LR_ERR_UNSUPPORTED),
+    (dict(shape=_shape(hidden=1024)), lr.LR_ERR_UNSUPPORTED),
+    (dict(shape=_shape(rank=0)), lr.LR_ERR_INVALID_ARG),
+    (dict(shape=_shape(T=-5)), lr.LR_ERR_INVALID_ARG),
+    (dict(shape=_shape(dtype=7)), lr.LR_ERR_INVALID_ARG),
+    (dict(pred=_pred(W1=None)), lr.LR_ERR_INVALID_ARG),
+    (dict(pred=_pred(per_sequence=2)), lr.LR_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments(lib, kw, status):
+    assert _decode(lib, **kw) == status
+    assert lib.lr_last_error()
+
+
+def test_null_shape_and_pack_checks(lib):
+    assert lib.lr_decode_attn(None, 0, 8, FAKE, FAKE, FAKE, None, None, None, None, 0, None, 0, 0.0, FAKE,
+                              FAKE, 1 << 40, None) == lr.LR_ERR_INVALID_ARG
+    shape, pred = _shape(), _pred()
+    args = [ctypes.byref(shape), FAKE, FAKE, FAKE, ctypes.byref(pred), 10, FAKE, FAKE, FAKE, None, None, FAKE]
+    assert lib.lr_pack_prefill(*args, 16, None) == lr.LR_ERR_WORKSPACE
+    bad = list(args)
+    bad[5] = 2000
+    assert lib.lr_pack_prefill(*bad, 1 << 40, None) == lr.LR_ERR_INVALID_ARG
+    bad = list(args)
+    bad[1] = None
+    assert lib.lr_pack_prefill(*bad, 1 << 40, None) == lr.LR_ERR_INVALID_ARG
+    assert lib.lr_topk_tokens(FAKE, 4, 100, 101, FAKE, FAKE, 256, None) == lr.LR_ERR_INVALID_ARG
+    assert lib.lr_topk_tokens(FAKE, 4, 100, 10, FAKE, FAKE, 16, None) == lr.LR_ERR_WORKSPACE
+    assert lib.lr_residual_block_ptr(FAKE, 4, 10, 100, None, None) == lr.LR_ERR_INVALID_ARG
+
+
+def test_workspace_sizes_grow_with_work(lib):
+    s1, s2 = _shape(T=1000), _shape(T=100000)
+    assert 0 < lib.lr_pack_workspace_bytes(ctypes.byref(s1), 10) < lib.lr_pack_workspace_bytes(ctypes.byref(s2), 10)
+    assert lib.lr_decode_workspace_bytes(ctypes.byref(s1), 8, 0) >= 256
+    assert lib.lr_decode_workspace_bytes(ctypes.byref(_shape(head_dim=12)), 8, 0) == 0

@@ -1,0 +1,135 @@
+"""GPU parity of lr_decode_attn against the fp64 oracle.
+
+Small cases span several 64-token blocks and a ragged tail and cover the
+degenerate cases (no residuals, a residual on every token, a single selected
+block, every block selected, an empty selection, T = 0 and T = 1, GQA 1..8,
+hidden 64..256, with and without block pointers, a nonzero b2). Full-size
+cases run the workloads of the benchmark in the launch configuration it times.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_lr_b200 import lowram as lr
+from long_context_decode_lr_b200 import synth
+
+import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from long_context_decode_lr_b200 import build
+    build.build()
+    lr.library()
+
+
+def _run(p, layer=1, **kw):
+    q_st, q_ref = H.queries(p, layer)
+    got, code = H.gpu_decode(p, layer, q_st, **kw)
+    ref = H.oracle_decode(p, layer, q_ref, scale=kw.get("scale", 0.0), blocks=kw.get("blocks"))
+    return got, ref, code
+
+
+def test_tiny_1k_fp32():
+    w = synth.WORKLOADS["tiny_1k"]
+    p = H.packed_problem(w)
+    got, ref, code = _run(p, layer=0)
+    assert code == 0
+    H.assert_attention_close(got, ref, rel_l2=1e-4, max_abs=1e-4)
+
+
+CASES = {
+    "ragged_full": dict(w=dict(q_per_kv=4, hidden=256, T=1000), sel=None, ptr=True),
+    "ragged_sel5": dict(w=dict(q_per_kv=4, hidden=256, T=1000), sel=5, ptr=True),
+    "gqa1_h64_noptr": dict(w=dict(q_per_kv=1, hidden=64, T=777), sel=None, ptr=False),
+    "gqa2_h128_sel3_noptr": dict(w=dict(q_per_kv=2, hidden=128, T=640), sel=3, ptr=False),
+    "gqa8_b2": dict(w=dict(q_per_kv=8, hidden=256, T=300), sel=None, ptr=True, b2=True),
+    "no_residuals": dict(w=dict(T=1000), k=0),
+    "residual_every_token": dict(w=dict(T=1000), k=1000),
+    "all_blocks_listed": dict(w=dict(T=1000), sel="all"),
+    "one_block": dict(w=dict(T=1000), sel=1),
+    "single_token": dict(w=dict(T=1, res_pct=100)),
+    "batch3": dict(w=dict(T=513, batch=3), sel=None),
+    "batch2_sel": dict(w=dict(T=900, batch=2), sel=4),
+    "hd64_rank64": dict(w=dict(head_dim=64, rank=64, hidden=128, T=700)),
+    "scale_given": dict(w=dict(T=400), scale=0.05),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_small_bf16(name):
+    c = CASES[name]
+    w = H.small(**c["w"])
+    p = H.packed_problem(w, k=c.get("k"), with_b2=c.get("b2", False), sel=c.get("sel"))
+    got, ref, code = _run(p, use_ptr=c.get("ptr", True), scale=c.get("scale", 0.0))
+    assert code == 0
+    H.assert_attention_close(got, ref)
+
+
+def test_ptr_and_search_agree():
+    w = H.small(T=1000)
+    p = H.packed_problem(w, sel=6)
+    q_st, _ = H.queries(p, 0)
+    a, _ = H.gpu_decode(p, 0, q_st, use_ptr=True)
+    b, _ = H.gpu_decode(p, 0, q_st, use_ptr=False)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_empty_selection_and_empty_context_give_zero():
+    w = H.small(T=640)
+    p = H.packed_problem(w, sel=2)
+    q_st, _ = H.queries(p, 0)
+    got, code = H.gpu_decode(p, 0, q_st, blocks=np.zeros((1, w.n_kv_heads, 0), np.int32), n_sel=0)
+    assert code == 0 and np.all(got == 0)
+    w0 = H.small(T=0, res_pct=0)
+    shape = H.shape_of(w0)
+    o = torch.full((1, w0.n_q_heads, w0.head_dim), 7.0, dtype=torch.bfloat16, device="cuda")
+    ws = lr.workspace(lr.lr_decode_workspace_bytes(shape, w0.n_q_heads, 0))
+    one = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    pred = lr.Predictor(p.st["W_lin"], p.st["W1"], p.st["b1"], p.st["W2"])
+    lr.lr_decode_attn(shape, 0, w0.n_q_heads, q_st, one, p.st["Bt"], pred, None, None, None, 0, None, 0, 0.0, o, ws)
+    assert lr.lr_get_device_error(ws) == 0
+    assert torch.all(o == 0)
+
+
+def test_bad_block_lists_set_the_error_word():
+    w = H.small(T=1000)
+    p = H.packed_problem(w, sel=4)
+    q_st, q_ref = H.queries(p, 0)
+    bad = p.blocks.copy()
+    bad[0, 0, 1], bad[0, 0, 2] = bad[0, 0, 2], bad[0, 0, 1]      # not ascending
+    bad[0, 1, 3] = w.nblk + 5                                      # out of range
+    got, code = H.gpu_decode(p, 0, q_st, blocks=bad)
+    assert code & lr.LR_DEVERR_BLOCK_ORDER and code & lr.LR_DEVERR_BLOCK_RANGE
+    assert np.all(np.isfinite(got))
+    # the rejected entries are skipped: head 1 attends to its first three blocks only
+    ref = H.oracle_decode(p, 0, q_ref, blocks=[[list(bad[0, 0, [0, 1, 3]]), list(bad[0, 1, :3])]])
+    H.assert_attention_close(got, ref)
+
+
+def test_bad_residual_pointers_set_the_error_word():
+    w = H.small(T=1000)
+    p = H.packed_problem(w)
+    p.st["ptr"][0, 1, 0, 3] = 10 ** 6
+    q_st, _ = H.queries(p, 1)
+    got, code = H.gpu_decode(p, 1, q_st)
+    assert code & lr.LR_DEVERR_PTR and np.all(np.isfinite(got))
+
+
+# ----------------------------------------------------------------------------- full size
+
+FULL = [("mistral_group_32k", None), ("mistral_group_131k_b4_sel8", "list"),
+        ("llama_262k_full", None), ("llama_262k_sel16", "list")]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,sel", FULL)
+def test_full_size(name, sel):
+    w = synth.WORKLOADS[name]
+    p = H.direct_problem(w, sel=w.n_sel if sel else None)
+    layer = w.n_layers - 1
+    got, ref, code = _run(p, layer=layer)
+    assert code == 0
+    H.assert_attention_close(got, ref)

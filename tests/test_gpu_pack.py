@@ -1,0 +1,168 @@
+"""GPU parity of lr_pack_prefill against the fp64 oracle.
+
+A, the per-token errors and the residual rows are floating results (relative L2
+<= 1e-2). The residual index set is compared exactly, except for tokens whose
+oracle error lies within a relative band of 2^-7 around the k-th largest oracle
+error, where fp32 and fp64 scores may legitimately order differently; the GPU set
+must also be the exact top-k of the GPU's own errors (ties to the lower index),
+and the block pointers must count it exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+from long_context_decode_lr_b200 import lowram as lr
+from long_context_decode_lr_b200 import synth
+from oracle import lowram_oracle as orc
+
+import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+BAND = 2.0 ** -7
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from long_context_decode_lr_b200 import build
+    build.build()
+    lr.library()
+
+
+def gpu_pack(p, k, with_ptr=True, with_err=True):
+    w = p.w
+    dt = H.TORCH_DT[w.dtype]
+    B, L, Hkv, T = w.batch, w.n_layers, w.n_kv_heads, w.T
+    shape = H.shape_of(w)
+    A = torch.empty((B, T, w.rank), dtype=dt, device="cuda")
+    idx = torch.full((B, L, Hkv, k), -1, dtype=torch.int32, device="cuda")
+    val = torch.empty((B, L, Hkv, k, w.head_dim), dtype=dt, device="cuda")
+    ptr = torch.empty((B, L, Hkv, w.nblk + 1), dtype=torch.int32, device="cuda") if with_ptr else None
+    err = torch.empty((B, L, Hkv, T), dtype=torch.float32, device="cuda") if with_err else None
+    ws = lr.workspace(lr.lr_pack_workspace_bytes(shape, k))
+    pred = H.gpu_predictor(p)
+    lr.lr_pack_prefill(shape, p.st["K"], p.st["V"], p.st["Bt"], pred, k, A, idx if k else None,
+                       val if k else None, ptr, err, ws)
+    assert lr.lr_get_device_error(ws) == 0
+    out = dict(A=A.to(torch.float64).cpu().numpy(), idx=idx.cpu().numpy().astype(np.int64),
+               val=val.to(torch.float64).cpu().numpy())
+    if with_ptr:
+        out["ptr"] = ptr.cpu().numpy()
+    if with_err:
+        out["err"] = err.cpu().numpy().astype(np.float64)
+    return out
+
+
+def check_valid_topk(e, sel, k):
+    """sel is the exact top-k of e by (e desc, index asc), ascending."""
+    assert len(sel) == k and np.all(np.diff(sel) > 0)
+    if k == 0 or k == len(e):
+        return
+    mask = np.zeros(len(e), bool)
+    mask[sel] = True
+    lo = e[mask].min()
+    hi = e[~mask].max()
+    assert lo >= hi
+    if lo == hi:  # ties at the boundary: every tied unselected token has a higher index
+        assert np.flatnonzero(~mask & (e == hi)).min() > np.flatnonzero(mask & (e == lo)).max()
+
+
+def compare(p, g, k):
+    w, ref = p.w, p.ref
+    assert H.rel_l2(g["A"], ref["A"]) <= 1e-2
+    band_total = 0
+    for b in range(w.batch):
+        for l in range(w.n_layers):
+            for h in range(w.n_kv_heads):
+                e_ref = ref["err"][b, l, h]
+                assert H.rel_l2(g["err"][b, l, h], e_ref) <= 1e-2
+                gi, ri = g["idx"][b, l, h], ref["idx"][b, l, h]
+                check_valid_topk(g["err"][b, l, h], gi, k)
+                if 0 < k < w.T:
+                    ek = np.sort(e_ref)[::-1][k - 1]
+                    differ = np.setxor1d(gi, ri)
+                    assert np.all(np.abs(e_ref[differ] - ek) <= BAND * ek), "index sets differ outside the band"
+                    band_total += differ.size
+                else:
+                    np.testing.assert_array_equal(gi, ri)
+                common, gpos, rpos = np.intersect1d(gi, ri, return_indices=True)
+                if common.size:
+                    assert H.rel_l2(g["val"][b, l, h][gpos], ref["val"][b, l, h][rpos]) <= 1e-2
+                nblk = w.nblk
+                np.testing.assert_array_equal(g["ptr"][b, l, h], np.searchsorted(gi, 64 * np.arange(nblk + 1)))
+    return band_total
+
+
+PACK_CASES = {
+    "ragged_bf16": dict(w=dict(T=1000), k=100),
+    "hidden64_gqa1": dict(w=dict(T=777, hidden=64, q_per_kv=1), k=77),
+    "batch2_b2": dict(w=dict(T=513, batch=2), k=51, b2=True),
+    "no_residuals": dict(w=dict(T=640), k=0),
+    "every_token": dict(w=dict(T=300), k=300),
+    "hd64": dict(w=dict(T=500, head_dim=64, rank=64, hidden=128), k=120),
+}
+
+
+@pytest.mark.parametrize("name", list(PACK_CASES))
+def test_pack_small(name):
+    c = PACK_CASES[name]
+    w = H.small(**c["w"])
+    p = H.packed_problem(w, k=c["k"], with_b2=c.get("b2", False))
+    g = gpu_pack(p, c["k"])
+    compare(p, g, c["k"])
+
+
+def test_pack_tiny_1k_fp32():
+    w = synth.WORKLOADS["tiny_1k"]
+    p = H.packed_problem(w)
+    g = gpu_pack(p, w.k)
+    compare(p, g, w.k)
+
+
+def test_pack_without_optional_outputs_matches():
+    w = H.small(T=700)
+    p = H.packed_problem(w, k=70)
+    a = gpu_pack(p, 70)
+    b = gpu_pack(p, 70, with_ptr=False, with_err=False)
+    np.testing.assert_array_equal(a["idx"], b["idx"])
+    np.testing.assert_array_equal(a["val"], b["val"])
+    np.testing.assert_array_equal(a["A"], b["A"])
+
+
+def test_pack_duplicated_rows_tie_to_lower_index():
+    w = H.small(T=600, n_layers=1)
+    p0 = H.packed_problem(w, k=60, dup_rows=40)
+    # choose k so that the boundary falls inside a duplicated pair (t, t+1)
+    e = p0.ref["err"][0, 0, 0]
+    t = 5 + 3 * 7
+    assert e[t] == e[t + 1]
+    k = int(np.sum(e > e[t])) + 1
+    p = H.packed_problem(w, k=k, dup_rows=40)
+    g = gpu_pack(p, k)
+    ge = g["err"][0, 0, 0]
+    assert ge[t] == ge[t + 1]
+    check_valid_topk(ge, g["idx"][0, 0, 0], k)
+    compare(p, g, k)
+
+
+@pytest.fixture(scope="module")
+def pack_131k():
+    w = synth.WORKLOADS["pack_131k_r10"]
+    return H.packed_problem(w, k=0, oracle=False)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("pct", [5, 10, 25])
+def test_pack_full_size(pack_131k, pct):
+    w = synth.WORKLOADS[f"pack_131k_r{pct}"]
+    base = pack_131k
+    k = w.k
+    ref = base.ref
+    oracle = orc.pack_sequence(ref["K"][0], ref["V"][0], ref["Bt"][0], ref["W_lin"][0], ref["W1"][0], ref["b1"][0],
+                               ref["W2"][0], None, k, w.dtype, w.n_kv_heads, w.head_dim)
+    p = H.Problem(w=w, st=base.st, ref=dict(ref, A=oracle["A"][None], idx=oracle["idx"][None],
+                                            val=oracle["val"][None], err=oracle["err"][None]),
+                  k=k, blocks=None, has_b2=False)
+    g = gpu_pack(p, k)
+    band = compare(p, g, k)
+    assert band <= 0.001 * k * w.n_layers * w.n_kv_heads
