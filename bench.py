@@ -215,6 +215,14 @@ def build_cache(w: synth.Workload, lr, seed_offset: int = 0):
                           "tflops": pack_flops / (pack_ms * 1e-3) / 1e12, "k": k}
 
 
+def decode_launches_per_step(w: synth.Workload, n_sel: int) -> int:
+    """Kernels one lr_decode_attn call launches (tensor-core path: W1 conversion, [schedule],
+    main kernel, combine; general path: main kernel, combine)."""
+    tc = (w.dtype == "bf16" and w.head_dim == 128 and w.hidden in (128, 256) and w.rank % 64 == 0
+          and w.n_kv_heads % 2 == 0 and w.q_per_kv <= 8 and w.T > 0)
+    return (3 + (1 if n_sel else 0)) if tc else 2
+
+
 def clone_cache(c, lr):
     d = {k: (v.clone() if isinstance(v, torch.Tensor) else [x.clone() for x in v]) for k, v in c.items()}
     d["pred"] = lr.Predictor(d["W_lin"], d["W1"], d["b1"], d["W2"], None, True)
@@ -327,7 +335,7 @@ def run_lowram(args, world, rank):
                 "h2d_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "d2h_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "ms_per_step": e2e_ms},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": decode_launches_per_step(w, n_sel) * args.steps,
         "clocks": clk.summary(),
         "pack": pack,
     }

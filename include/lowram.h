@@ -71,6 +71,7 @@ typedef enum lr_dtype { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
 #define LR_DEVERR_RES_RANGE 4   /* a residual index outside its block or [0, T): entry skipped */
 #define LR_DEVERR_RES_ORDER 8   /* residual indices not strictly ascending */
 #define LR_DEVERR_PTR 16        /* a residual block pointer out of [0, k] or decreasing */
+#define LR_DEVERR_TIMEOUT 32    /* a kernel gave up waiting on its own pipeline (its output is invalid) */
 
 typedef struct lr_cache_shape {
   int32_t batch;      /* B >= 0 */
@@ -79,7 +80,7 @@ typedef struct lr_cache_shape {
   int32_t n_kv_heads; /* Hkv >= 1 */
   int32_t head_dim;   /* hd: multiple of 8, <= 256 */
   int32_t rank;       /* r: multiple of 8, >= 8 */
-  int32_t hidden;     /* H: predictor hidden width, multiple of 8, <= 1024 */
+  int32_t hidden;     /* H: predictor hidden width, multiple of 8, <= 512 */
   lr_dtype dtype;     /* storage type of every floating tensor */
 } lr_cache_shape;
 

@@ -1,0 +1,705 @@
+// Tensor-core decode over the compressed cache (bf16, head_dim 128, sm_100a).
+//
+// One CTA owns (split, KV-head pair, sequence) and walks 128-token tiles (two
+// 64-token blocks: consecutive blocks in full mode, entries of the pair's
+// selected-block union in selective mode). Per tile:
+//   MMA1  S1[128 x 256]  = A_tile[128 x r] . [B_l^a | B_l^b]^T   (keys of both heads:
+//                          "LowRAM" project page, Figure 3)
+//   epilogue  scores q.k~ in fp32 from TMEM, k~ -> fp16 tile in shared memory,
+//             online softmax -> p (fp16 tile)
+//   MMA2  U[128 x 128]   = k~ . W1_half^T          (GELU branch input, per 128 hidden)
+//   epilogue  g = GELU(U + b1) -> fp16 tile         ("Predicting the value cache from
+//                                                     keys", paragraphs 2-3)
+//   MMA3  O3 += g^T . p, k~^T . p                   (p-weighted sums, fp32 in TMEM)
+//   epilogue  merge O3 into register accumulators with the softmax rescale and add
+//             p r over the tile's residual rows     (paragraph 2)
+// The second-stage operands (k~, g, p and W1) are fp16: 11 significant bits keep the
+// rebuilt values within the attention tolerance even when one token dominates.
+// Roles: warp 0 issues TMA loads into a 3-stage ring (A and B_l chunks of 64 rank
+// columns, then W1 halves), warp 1 issues the MMAs, warps 2-5 run the epilogue.
+// The split partials (m, l, sum p k~, sum p g, sum p r) go to the same combine
+// kernel as the general path. Every wait is bounded: on a timeout the CTA records
+// LR_DEVERR_TIMEOUT, drains what it issued and returns.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "lr_common.cuh"
+#include "lr_launch.h"
+#include "lr_tc.h"
+#include "sm100.cuh"
+
+namespace lr {
+namespace tc {
+namespace {
+
+using namespace sm100;
+
+constexpr int kHd = 128;
+constexpr int kChunk = 64;                 // rank columns per ring stage
+constexpr int kStages = 3;
+constexpr uint32_t kStageBytes = 48 * 1024;  // A rows 2 x 8 KB + B_l rows 2 x 16 KB
+constexpr int kThreads = 192;
+constexpr int kEpi = 128;
+
+constexpr uint32_t kColS1 = 0;
+constexpr uint32_t kColU = 256;
+constexpr uint32_t kColO3 = 384;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kOffRing = 0;
+constexpr uint32_t kOffKt = kStages * kStageBytes;
+constexpr uint32_t kOffG = kOffKt + 32768;
+constexpr uint32_t kOffP = kOffG + 32768;
+constexpr uint32_t kOffQ = kOffP + 4096;
+constexpr uint32_t kOffB1 = kOffQ + 8192;
+constexpr uint32_t kOffRed = kOffB1 + 2048;
+constexpr uint32_t kOffBar = kOffRed + 256;
+constexpr uint32_t kOffMisc = kOffBar + 256;
+constexpr uint32_t kSmemUsed = kOffMisc + 64;
+constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
+
+enum Bar {
+  FULL0 = 0, EMPTY0 = kStages, S1_FULL = 2 * kStages, S1_FREE, KT_READY, KT_FREE, U_FULL, U_FREE,
+  G_READY, G_FREE, O3_FULL0, O3_FULL1, O3_FREE0, O3_FREE1, DRAIN, EPI_SYNC, N_BARS
+};
+static_assert(N_BARS * 8 <= 256, "barrier area");
+
+// GELU(x) = x Phi(x) with Phi(x) ~ (1 + tanh(x (c1 + c3 x^2 + c5 x^4 + c7 x^6))) / 2, x
+// clamped to [-6, 6] inside tanh. Coefficients are a minimax fit to the exact erf form
+// (max abs error 1.2e-5 in exact arithmetic; csrc/gelu_fit.py reproduces them).
+constexpr float kG1 = 7.97690120e-01f, kG3 = 3.67308140e-02f, kG5 = -2.55099297e-04f, kG7 = -8.60763669e-06f;
+
+__device__ __forceinline__ float gelu_tc(float x) {
+  const float c = fminf(fmaxf(x, -6.f), 6.f);
+  const float s = c * c;
+  const float z = c * fmaf(s, fmaf(s, fmaf(s, kG7, kG5), kG3), kG1);
+  const float h = 0.5f * x;
+  return fmaf(h, tanh_fast(z), h);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+struct TileInfo {
+  int blk[2];
+  int mask[2];
+};
+
+__device__ __forceinline__ int tile_count(const TcArgs& a, int b, int hp) {
+  if (!a.sched) return (a.nblk + 1) >> 1;
+  return (a.sched[((size_t)b * a.n_hp + hp) * a.sched_stride] + 1) >> 1;
+}
+
+__device__ __forceinline__ TileInfo tile_info(const TcArgs& a, int b, int hp, int i) {
+  TileInfo t;
+  if (!a.sched) {
+    t.blk[0] = 2 * i;
+    t.blk[1] = 2 * i + 1 < a.nblk ? 2 * i + 1 : -1;
+    t.mask[0] = 3;
+    t.mask[1] = t.blk[1] >= 0 ? 3 : 0;
+    return t;
+  }
+  const int* s = a.sched + ((size_t)b * a.n_hp + hp) * a.sched_stride;
+  const int n = s[0];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = 2 * i + h;
+    if (e < n) {
+      const int v = s[1 + e];
+      t.blk[h] = v & 0x0FFFFFFF;
+      t.mask[h] = (v >> 28) & 3;
+    } else {
+      t.blk[h] = -1;
+      t.mask[h] = 0;
+    }
+  }
+  return t;
+}
+
+__device__ __forceinline__ int lower_bound_i32(const int* p, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (p[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// byte offset of element (row, col) of a 128-byte-swizzled 16-bit tile whose 64-column
+// atoms are `atom_bytes` apart
+__device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t atom_bytes) {
+  const int a = col >> 6, c = col & 63;
+  return a * atom_bytes + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + ((c & 7) << 1);
+}
+
+template <int MG>
+struct HeadState {
+  float m[MG], l[MG], ak[MG], ag0[MG], ag1[MG], ar[MG];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      m[g] = -CUDART_INF_F;
+      l[g] = ak[g] = ag0[g] = ag1[g] = ar[g] = 0.f;
+    }
+  }
+};
+
+struct EpiCtx {
+  int lq, ew, lane, row, tl, rmask;
+  uint32_t sync_phase;  // completed phases of the EPI_SYNC barrier
+  bool row_valid;
+  uint32_t trow;
+  uint8_t* sm;
+  uint64_t* bars;
+  volatile int* abort_flag;
+  size_t pseg;  // (b, layer, first head of the pair) segment index
+  TileInfo t;
+};
+
+// Epilogue-side wait: every lane polls, and the outcome is made uniform across the
+// warp so that a timeout never leaves part of a warp inside a collective.
+__device__ __forceinline__ bool ewait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+// Barrier over the four epilogue warps, bounded like every other wait.
+__device__ __forceinline__ bool epi_sync(EpiCtx& c) {
+  mbar_arrive(&c.bars[EPI_SYNC]);
+  const bool ok = ewait(&c.bars[EPI_SYNC], c.sync_phase & 1, c.abort_flag);
+  ++c.sync_phase;
+  return ok;
+}
+
+// The epilogue's work for one KV head (slot HX of the pair) on the current tile.
+template <int HX, int MG>
+__device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<MG>& st) {
+  const int G = a.G, nh = a.H / 128;
+  uint64_t* bars = c.bars;
+  const float* qs = reinterpret_cast<const float*>(c.sm + kOffQ);
+  const float* b1s = reinterpret_cast<const float*>(c.sm + kOffB1);
+  float* red = reinterpret_cast<float*>(c.sm + kOffRed);
+  uint8_t* ktile = c.sm + kOffKt;
+  uint8_t* gtile = c.sm + kOffG;
+  uint8_t* ptile = c.sm + kOffP;
+  const int row = c.row, lane = c.lane;
+  const int n_kt = 2 * c.tl + HX;
+  if (n_kt > 0 && !ewait(&bars[KT_FREE], (n_kt - 1) & 1, c.abort_flag)) return false;
+  // ---- scores and the fp16 key tile
+  float sc[MG];
+#pragma unroll
+  for (int g = 0; g < MG; ++g) sc[g] = 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t v[32];
+    tmem_ld32(c.trow + kColS1 + HX * 128 + cc * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      if (g < G) {
+        const float4* q4 = reinterpret_cast<const float4*>(qs + (HX * 8 + g) * kHd + cc * 32);
+        float acc = sc[g];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float4 qq = q4[j];
+          acc = fmaf(__uint_as_float(v[4 * j]), qq.x, acc);
+          acc = fmaf(__uint_as_float(v[4 * j + 1]), qq.y, acc);
+          acc = fmaf(__uint_as_float(v[4 * j + 2]), qq.z, acc);
+          acc = fmaf(__uint_as_float(v[4 * j + 3]), qq.w, acc);
+        }
+        sc[g] = acc;
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 w;
+      w.x = pack_f16x2_sat(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+      w.y = pack_f16x2_sat(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+      w.z = pack_f16x2_sat(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+      w.w = pack_f16x2_sat(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+      *reinterpret_cast<uint4*>(ktile + sw128_off(row, cc * 32 + q * 8, 16384)) = w;
+    }
+  }
+  if (HX == 1) {
+    tc_fence_before();
+    mbar_arrive(&bars[S1_FREE]);
+  }
+  // ---- online softmax over the tile
+  const bool hv = c.row_valid && ((c.rmask >> HX) & 1);
+  float alpha[MG], p[MG];
+#pragma unroll
+  for (int g = 0; g < MG; ++g) {
+    if (!hv) sc[g] = -CUDART_INF_F;
+    const float m = warp_max(sc[g]);
+    if (lane == 0) red[c.ew * 16 + g] = m;
+  }
+  if (!epi_sync(c)) return false;
+#pragma unroll
+  for (int g = 0; g < MG; ++g) {
+    const float mt = fmaxf(fmaxf(red[g], red[16 + g]), fmaxf(red[32 + g], red[48 + g]));
+    const float m_new = fmaxf(st.m[g], mt);
+    alpha[g] = m_new == -CUDART_INF_F ? 1.f : __expf(st.m[g] - m_new);
+    p[g] = hv ? __expf(sc[g] - m_new) : 0.f;
+    st.l[g] = st.l[g] * alpha[g] + p[g];
+    st.m[g] = m_new;
+  }
+#pragma unroll
+  for (int g = 0; g < MG; ++g)
+    if (g < G) *reinterpret_cast<__half*>(ptile + sw128_off(g, row, 2048)) = __float2half_rn(p[g]);
+  fence_proxy_async_smem();
+  if (!epi_sync(c)) return false;  // p tile complete (read back below) and red consumed
+  mbar_arrive(&bars[KT_READY]);
+  // ---- GELU branch, one 128-unit half at a time
+#pragma unroll 1
+  for (int half = 0; half < nh; ++half) {
+    const int j = n_kt * nh + half;
+    if (!ewait(&bars[U_FULL], j & 1, c.abort_flag)) return false;
+    tc_fence_after();
+    uint32_t u[4][32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld32(c.trow + kColU + q * 32, u[q]);
+    tmem_ld_wait();
+    tc_fence_before();
+    mbar_arrive(&bars[U_FREE]);
+    if (j > 0 && !ewait(&bars[G_FREE], (j - 1) & 1, c.abort_flag)) return false;
+    const float* bb = b1s + HX * 256 + half * 128;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int col = q * 8;
+      const uint32_t* uu = &u[q >> 2][(q & 3) * 8];
+      uint4 w;
+      w.x = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[0]) + bb[col + 0]), gelu_tc(__uint_as_float(uu[1]) + bb[col + 1]));
+      w.y = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[2]) + bb[col + 2]), gelu_tc(__uint_as_float(uu[3]) + bb[col + 3]));
+      w.z = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[4]) + bb[col + 4]), gelu_tc(__uint_as_float(uu[5]) + bb[col + 5]));
+      w.w = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[6]) + bb[col + 6]), gelu_tc(__uint_as_float(uu[7]) + bb[col + 7]));
+      *reinterpret_cast<uint4*>(gtile + sw128_off(row, col, 16384)) = w;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars[G_READY]);
+  }
+  // ---- merge this tile's p-weighted sums (O3 lane = dim `row`)
+  if (!ewait(&bars[O3_FULL0 + HX], c.tl & 1, c.abort_flag)) return false;
+  tc_fence_after();
+  uint32_t ok8[8], og0[8], og1[8];
+  tmem_ld8(c.trow + kColO3 + HX * 48, ok8);
+  tmem_ld8(c.trow + kColO3 + HX * 48 + 16, og0);
+  tmem_ld8(c.trow + kColO3 + HX * 48 + 32, og1);
+  tmem_ld_wait();
+  tc_fence_before();
+  mbar_arrive(&bars[O3_FREE0 + HX]);
+#pragma unroll
+  for (int g = 0; g < MG; ++g) {
+    st.ak[g] = fmaf(st.ak[g], alpha[g], __uint_as_float(ok8[g]));
+    st.ag0[g] = fmaf(st.ag0[g], alpha[g], __uint_as_float(og0[g]));
+    st.ag1[g] = fmaf(st.ag1[g], alpha[g], __uint_as_float(og1[g]));
+    st.ar[g] *= alpha[g];
+  }
+  // ---- residual rows of the tile's blocks: ar += p_t r_t[dim]
+  if (a.k > 0) {
+    const size_t seg = c.pseg + HX;
+    const int* ridx = a.res_idx + seg * a.k;
+    const __nv_bfloat16* rval = a.res_val + seg * a.k * kHd;
+    const int* rptr = a.res_ptr ? a.res_ptr + seg * (a.nblk + 1) : nullptr;
+#pragma unroll 1
+    for (int bh = 0; bh < 2; ++bh) {
+      const int blk = c.t.blk[bh];
+      if (blk < 0 || !((c.t.mask[bh] >> HX) & 1)) continue;
+      int e0, e1;
+      if (rptr) {
+        e0 = rptr[blk];
+        e1 = rptr[blk + 1];
+        if (e0 < 0 || e1 < e0 || e1 > a.k) {
+          if (row == 0) flag_error(a.err, LR_DEVERR_PTR);
+          continue;
+        }
+      } else {
+        e0 = lower_bound_i32(ridx, a.k, blk * kBlock);
+        e1 = lower_bound_i32(ridx, a.k, blk * kBlock + kBlock);
+      }
+      const int lo = blk * kBlock, hi = min(lo + kBlock, a.T);
+#pragma unroll 1
+      for (int e = e0; e < e1; ++e) {
+        const int tr = ridx[e];
+        if (tr < lo || tr >= hi) {
+          if (row == 0) flag_error(a.err, LR_DEVERR_RES_RANGE);
+          continue;
+        }
+        if (e > e0 && ridx[e - 1] >= tr && row == 0) flag_error(a.err, LR_DEVERR_RES_ORDER);
+        const float rv = __bfloat162float(rval[(size_t)e * kHd + row]);
+        const int prow = bh * 64 + (tr - lo);
+#pragma unroll
+        for (int g = 0; g < MG; ++g) {
+          if (g < G) {
+            const float pg = __half2float(*reinterpret_cast<const __half*>(ptile + sw128_off(g, prow, 2048)));
+            st.ar[g] = fmaf(pg, rv, st.ar[g]);
+          }
+        }
+      }
+    }
+  }
+  return true;
+}
+
+template <int MG>
+__device__ __forceinline__ void write_partials(const TcArgs& a, EpiCtx& c, const HeadState<MG>& s0,
+                                               const HeadState<MG>& s1, int b, int split, int ha) {
+  float* red = reinterpret_cast<float*>(c.sm + kOffRed);
+  epi_sync(c);  // red is free
+#pragma unroll
+  for (int g = 0; g < MG; ++g) {
+    const float v0 = warp_sum(s0.l[g]);
+    const float v1 = warp_sum(s1.l[g]);
+    if (c.lane == 0) {
+      red[c.ew * 16 + g] = v0;
+      red[c.ew * 16 + 8 + g] = v1;
+    }
+  }
+  epi_sync(c);
+  const int Hq = a.Hkv * a.G, row = c.row;
+#pragma unroll
+  for (int hx = 0; hx < 2; ++hx) {
+    const HeadState<MG>& st = hx ? s1 : s0;
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      if (g >= a.G) continue;
+      const int hq = (ha + hx) * a.G + g;
+      float* part = a.partials + (((size_t)b * Hq + hq) * a.n_split + split) * a.part_stride;
+      if (row == 0) {
+        part[0] = st.m[g];
+        part[1] = red[hx * 8 + g] + red[16 + hx * 8 + g] + red[32 + hx * 8 + g] + red[48 + hx * 8 + g];
+        part[2] = part[3] = 0.f;
+      }
+      part[4 + row] = st.ak[g];
+      part[4 + kHd + row] = st.ag0[g];
+      if (a.H == 256) part[4 + kHd + 128 + row] = st.ag1[g];
+      part[4 + kHd + a.H + row] = st.ar[g];
+    }
+  }
+}
+
+template <int MG>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                 const __grid_constant__ CUtensorMap mapW1, const TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+
+  const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.G, H = a.H, nh = a.H / 128, nk = a.r / kChunk;
+  const int n_tiles = tile_count(a, b, hp);
+  const int t_begin = (int)((long long)s * n_tiles / a.n_split);
+  const int t_end = (int)((long long)(s + 1) * n_tiles / a.n_split);
+  const int ha = 2 * hp;  // first KV head of the pair
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&bars[FULL0 + i], 1);
+      mbar_init(&bars[EMPTY0 + i], 1);
+    }
+    mbar_init(&bars[S1_FULL], 1);
+    mbar_init(&bars[S1_FREE], kEpi);
+    mbar_init(&bars[KT_READY], kEpi);
+    mbar_init(&bars[KT_FREE], 1);
+    mbar_init(&bars[U_FULL], 1);
+    mbar_init(&bars[U_FREE], kEpi);
+    mbar_init(&bars[G_READY], kEpi);
+    mbar_init(&bars[G_FREE], 1);
+    mbar_init(&bars[O3_FULL0], 1);
+    mbar_init(&bars[O3_FULL1], 1);
+    mbar_init(&bars[O3_FREE0], kEpi);
+    mbar_init(&bars[O3_FREE1], kEpi);
+    mbar_init(&bars[DRAIN], 1);
+    mbar_init(&bars[EPI_SYNC], kEpi);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapA);
+    tma_prefetch_desc(&mapB);
+    tma_prefetch_desc(&mapW1);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
+  }
+  {  // query rows of the pair (pre-scaled), b1 of both heads, zero p tile
+    float* qs = reinterpret_cast<float*>(sm + kOffQ);
+    const __nv_bfloat16* q = a.q + ((size_t)b * a.Hkv * G + (size_t)ha * G) * kHd;
+    for (int i = threadIdx.x; i < 2 * 8 * kHd; i += kThreads) {
+      const int hx = i / (8 * kHd), g = (i / kHd) % 8, d = i % kHd;
+      qs[i] = g < G ? __bfloat162float(q[((size_t)hx * G + g) * kHd + d]) * a.scale : 0.f;
+    }
+    float* b1s = reinterpret_cast<float*>(sm + kOffB1);
+    const size_t pseq = a.pred_per_seq ? (size_t)b : 0;
+    for (int i = threadIdx.x; i < 2 * 256; i += kThreads) {
+      const int hx = i / 256, c = i % 256;
+      b1s[i] = c < H ? __bfloat162float(a.b1[((pseq * a.L + a.layer) * a.Hkv + ha + hx) * H + c]) : 0.f;
+    }
+    uint32_t* pz = reinterpret_cast<uint32_t*>(sm + kOffP);
+    for (int i = threadIdx.x; i < 1024; i += kThreads) pz[i] = 0u;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      const int rowB = (a.layer * a.Hkv + ha) * kHd;
+      const int w1seq = a.pred_per_seq ? b : 0;
+      for (int ti = t_begin; ti < t_end && ok; ++ti) {
+        const TileInfo t = tile_info(a, b, hp, ti);
+        const int row0 = t.blk[0] >= 0 ? t.blk[0] * kBlock : a.T;
+        const int row1 = t.blk[1] >= 0 ? t.blk[1] * kBlock : a.T;
+        for (int kc = 0; kc < nk && ok; ++kc, ++it) {
+          const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+          if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
+          uint8_t* dst = sm + kOffRing + st * kStageBytes;
+          mbar_arrive_expect_tx(&bars[FULL0 + st], kStageBytes);
+          tma_load_3d(dst, &mapA, &bars[FULL0 + st], kc * kChunk, row0, b);
+          tma_load_3d(dst + 8192, &mapA, &bars[FULL0 + st], kc * kChunk, row1, b);
+          tma_load_3d(dst + 16384, &mapB, &bars[FULL0 + st], kc * kChunk, rowB, b);
+          tma_load_3d(dst + 32768, &mapB, &bars[FULL0 + st], kc * kChunk, rowB + kHd, b);
+        }
+        for (int hx = 0; hx < 2 && ok; ++hx) {
+          for (int half = 0; half < nh && ok; ++half, ++it) {
+            const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+            if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
+            uint8_t* dst = sm + kOffRing + st * kStageBytes;
+            const int wrow = ((w1seq * a.Hkv + ha + hx) * H) + half * 128;
+            mbar_arrive_expect_tx(&bars[FULL0 + st], 32768);
+            tma_load_2d(dst, &mapW1, &bars[FULL0 + st], 0, wrow);
+            tma_load_2d(dst + 16384, &mapW1, &bars[FULL0 + st], 64, wrow);
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(a.err, LR_DEVERR_TIMEOUT);
+      }
+      // drain: every load issued has landed before the CTA may exit
+      for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+        mbar_wait_drain(&bars[FULL0 + j % kStages], (j / kStages) & 1, kWaitCycles / 4);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s1 = idesc_bf16_f32(128, 256, false, false);
+      const uint32_t id_u = idesc_f16_f32(128, 128, false, false);
+      const uint32_t id_o3 = idesc_f16_f32(128, 16, true, false);
+      const uint32_t kt = smem_u32(sm + kOffKt), gt = smem_u32(sm + kOffG), pt = smem_u32(sm + kOffP);
+      uint32_t it = 0;
+      bool ok = true;
+      int tl = 0;
+      for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
+        if (!(ok = mbar_wait(&bars[S1_FREE], (tl & 1) ^ 1, abort_flag))) break;
+        tc_fence_after();
+        for (int kc = 0; kc < nk && ok; ++kc, ++it) {
+          const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+          if (!(ok = mbar_wait(&bars[FULL0 + st], ph, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t base = smem_u32(sm + kOffRing + st * kStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_f16_ss(tmem + kColS1, sw128_desc(base + ks * 32, 16, 1024),
+                        sw128_desc(base + 16384 + ks * 32, 16, 1024), id_s1, (kc | ks) != 0);
+          mma_commit(&bars[EMPTY0 + st]);
+        }
+        if (!ok) break;
+        mma_commit(&bars[S1_FULL]);
+        for (int hx = 0; hx < 2 && ok; ++hx) {
+          const int n_kt = 2 * tl + hx;
+          if (!(ok = mbar_wait(&bars[KT_READY], n_kt & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(&bars[O3_FREE0 + hx], (tl & 1) ^ 1, abort_flag))) break;
+          tc_fence_after();
+          for (int half = 0; half < nh && ok; ++half, ++it) {
+            const int j = n_kt * nh + half;
+            const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+            if (!(ok = mbar_wait(&bars[FULL0 + st], ph, abort_flag))) break;
+            if (!(ok = mbar_wait(&bars[U_FREE], (j & 1) ^ 1, abort_flag))) break;
+            tc_fence_after();
+            const uint32_t wb = smem_u32(sm + kOffRing + st * kStageBytes);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
+              mma_f16_ss(tmem + kColU, sw128_desc(kt + off, 16, 1024), sw128_desc(wb + off, 16, 1024), id_u,
+                          ks != 0);
+            }
+            mma_commit(&bars[EMPTY0 + st]);
+            mma_commit(&bars[U_FULL]);
+          }
+          for (int half = 0; half < nh && ok; ++half) {
+            const int j = n_kt * nh + half;
+            if (!(ok = mbar_wait(&bars[G_READY], j & 1, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              mma_f16_ss(tmem + kColO3 + hx * 48 + 16 + half * 16, sw128_desc(gt + ks * 2048, 16384, 1024),
+                          sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
+            mma_commit(&bars[G_FREE]);
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16_ss(tmem + kColO3 + hx * 48, sw128_desc(kt + ks * 2048, 16384, 1024),
+                        sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
+          mma_commit(&bars[KT_FREE]);
+          mma_commit(&bars[O3_FULL0 + hx]);
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        flag_error(a.err, LR_DEVERR_TIMEOUT);
+      }
+      // every MMA issued has completed before TMEM is released
+      mma_commit(&bars[DRAIN]);
+      mbar_wait_drain(&bars[DRAIN], 0, kWaitCycles / 4);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    EpiCtx c;
+    c.lq = warp & 3;
+    c.ew = warp - 2;
+    c.lane = lane;
+    c.row = c.lq * 32 + lane;
+    c.trow = tmem + ((uint32_t)(c.lq * 32) << 16);
+    c.sm = sm;
+    c.bars = bars;
+    c.abort_flag = abort_flag;
+    c.sync_phase = 0;
+    c.pseg = ((size_t)b * a.L + a.layer) * a.Hkv + ha;
+    HeadState<MG> st0, st1;
+    st0.init();
+    st1.init();
+    bool ok = true;
+    int tl = 0;
+    for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
+      c.t = tile_info(a, b, hp, ti);
+      const int half_row = c.row >> 6;
+      const int rblk = c.t.blk[half_row];
+      const int tok = rblk * kBlock + (c.row & 63);
+      c.row_valid = rblk >= 0 && tok < a.T;
+      c.rmask = c.t.mask[half_row];
+      c.tl = tl;
+      if (!(ok = ewait(&bars[S1_FULL], tl & 1, abort_flag))) break;
+      tc_fence_after();
+      ok = epi_head<0, MG>(a, c, st0);
+      if (ok) ok = epi_head<1, MG>(a, c, st1);
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      flag_error(a.err, LR_DEVERR_TIMEOUT);
+    }
+    write_partials(a, c, st0, st1, b, s, ha);
+  }
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// The layer's W1 as fp16 (the second-stage MMAs take fp16 operands so that the rebuilt
+// keys and GELU outputs keep 11 significant bits). bf16 -> fp16 is exact except for
+// magnitudes below 2^-14 (fp16 subnormals) or above 65504 (saturated).
+__global__ void decode_tc_w1_kernel(TcArgs a) {
+  const size_t per_seq = (size_t)a.Hkv * a.H * kHd;
+  const size_t n = (size_t)a.w1_seqs * per_seq;
+  for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n; i += (size_t)gridDim.x * blockDim.x * 4) {
+    const size_t sq = i / per_seq, r = i % per_seq;
+    const __nv_bfloat16* src = a.W1 + (sq * a.L + a.layer) * per_seq + r;
+    const uint2 v = *reinterpret_cast<const uint2*>(src);
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+    uint2 o;
+    o.x = pack_f16x2_sat(__low2float(lo), __high2float(lo));
+    o.y = pack_f16x2_sat(__low2float(hi), __high2float(hi));
+    *reinterpret_cast<uint2*>(a.W1h + i) = o;
+  }
+}
+
+// Per (sequence, KV-head pair): merge the two selected-block lists into one ascending
+// union with a 2-bit head mask per block (bit 0: first head, bit 1: second). Entries that
+// are out of range or not strictly ascending are skipped and flagged.
+__global__ void decode_tc_schedule_kernel(TcArgs a, const int* __restrict__ blocks, int n_sel, int* sched) {
+  const int hp = blockIdx.x, b = blockIdx.y;
+  if (threadIdx.x != 0) return;
+  const int* la = blocks + ((size_t)b * a.Hkv + 2 * hp) * n_sel;
+  const int* lb = la + n_sel;
+  int* out = sched + ((size_t)b * a.n_hp + hp) * a.sched_stride;
+  int i = 0, j = 0, n = 0, prev_a = -1, prev_b = -1, bits = 0;
+  auto next = [&](const int* l, int& k, int& prev) -> int {
+    while (k < n_sel) {
+      const int v = l[k];
+      const bool bad_range = v < 0 || v >= a.nblk;
+      const bool bad_order = k > 0 && l[k - 1] >= v;
+      if (bad_range) bits |= LR_DEVERR_BLOCK_RANGE;
+      if (bad_order) bits |= LR_DEVERR_BLOCK_ORDER;
+      if (!bad_range && !bad_order && v > prev) return v;
+      ++k;
+    }
+    return -1;
+  };
+  int va = next(la, i, prev_a), vb = next(lb, j, prev_b);
+  while (va >= 0 || vb >= 0) {
+    int v, m;
+    if (vb < 0 || (va >= 0 && va < vb)) { v = va; m = 1; prev_a = va; ++i; }
+    else if (va < 0 || vb < va) { v = vb; m = 2; prev_b = vb; ++j; }
+    else { v = va; m = 3; prev_a = va; prev_b = vb; ++i; ++j; }
+    out[1 + n++] = v | (m << 28);
+    va = next(la, i, prev_a);
+    vb = next(lb, j, prev_b);
+  }
+  out[0] = n;
+  if (bits) flag_error(a.err, bits);
+}
+
+}  // namespace
+
+size_t decode_tc_smem_bytes() { return kSmemBytes; }
+
+cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mW1,
+                             const int* blocks, int n_sel, cudaStream_t st) {
+  cudaError_t e;
+  {
+    const size_t n = (size_t)a.w1_seqs * a.Hkv * a.H * kHd / 4;
+    const int blocks_w1 = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+    decode_tc_w1_kernel<<<blocks_w1, 256, 0, st>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.sched) {
+    decode_tc_schedule_kernel<<<dim3(a.n_hp, a.B), 32, 0, st>>>(a, blocks, n_sel, const_cast<int*>(a.sched));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const dim3 grid(a.n_split, a.n_hp, a.B);
+  if (a.G <= 4) {
+    e = cudaFuncSetAttribute(decode_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<4><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, mW1, a);
+  } else {
+    e = cudaFuncSetAttribute(decode_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    decode_tc_kernel<8><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, mW1, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+}  // namespace lr

@@ -19,6 +19,7 @@ struct DecodePlan {
   int part_stride;   // floats per split partial
   size_t part_off;   // byte offset of the partials in the workspace
   size_t sched_off;  // byte offset of the tensor path's block schedule
+  size_t w1h_off;    // byte offset of the tensor path's fp16 copy of the layer's W1
   size_t ws_bytes;   // total workspace
 };
 
@@ -29,6 +30,7 @@ struct PackPlan {
   size_t ws_bytes;
 };
 
+bool decode_tc_supported(const lr_cache_shape& s, int n_q_heads);
 DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);
 PackPlan plan_pack(const lr_cache_shape& s, int k);
 

@@ -1,0 +1,39 @@
+// Internal interface of the tensor-core decode kernel.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace lr {
+namespace tc {
+
+struct TcArgs {
+  int B, T, L, Hkv, G, H, r;
+  int layer, k, nblk, pred_per_seq;
+  int n_hp;          // KV-head pairs
+  int n_split;       // CTAs per (sequence, head pair)
+  float scale;
+  const __nv_bfloat16* q;        // [B, Hq, 128]
+  const __nv_bfloat16* b1;       // [(B,) L, Hkv, H]
+  const __nv_bfloat16* W1;       // [(B,) L, Hkv, H, 128]
+  __half* W1h;                   // workspace: [(B,) Hkv, H, 128] fp16 copy of the layer's W1
+  int w1_seqs;                   // 1, or B when each sequence has its own predictor
+  const int* res_idx;            // [B, L, Hkv, k]
+  const __nv_bfloat16* res_val;  // [B, L, Hkv, k, 128]
+  const int* res_ptr;            // [B, L, Hkv, nblk + 1] or null
+  const int* sched;              // selective mode: [B, n_hp, sched_stride]; null in full mode
+  int sched_stride;              // 1 + 2 * n_sel
+  float* partials;               // [B, Hq, n_split, part_stride]
+  int part_stride;
+  int* err;
+};
+
+size_t decode_tc_smem_bytes();
+cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mW1,
+                             const int* blocks, int n_sel, cudaStream_t st);
+
+}  // namespace tc
+}  // namespace lr
