@@ -216,11 +216,11 @@ def build_cache(w: synth.Workload, lr, seed_offset: int = 0):
 
 
 def decode_launches_per_step(w: synth.Workload, n_sel: int) -> int:
-    """Kernels one lr_decode_attn call launches (tensor-core path: W1 conversion, [schedule],
-    main kernel, combine; general path: main kernel, combine)."""
+    """Kernels one lr_decode_attn call launches (tensor-core path: prep, main kernel, combine;
+    general path: main kernel, combine)."""
     tc = (w.dtype == "bf16" and w.head_dim == 128 and w.hidden in (128, 256) and w.rank % 64 == 0
           and w.n_kv_heads % 2 == 0 and w.q_per_kv <= 8 and w.T > 0)
-    return (3 + (1 if n_sel else 0)) if tc else 2
+    return 3 if tc else 2
 
 
 def clone_cache(c, lr):

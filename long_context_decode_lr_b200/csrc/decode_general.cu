@@ -160,53 +160,77 @@ __global__ void __launch_bounds__(NT) decode_general_kernel(DecodeArgs a) {
   }
 }
 
-// Merge the split partials of one (sequence, query head) and apply the linear maps.
+// Merge the split partials of the G query heads of one (sequence, KV head) and apply
+// the linear maps once per query head: o = (acc_k W_lin^T + acc_g W2^T + acc_r) / l + b2.
+// Partial sums are read coalesced (threads over entries); each output element is a
+// warp-wide dot product over a contiguous weight row.
+constexpr int CT = 512;  // combine threads
+
 template <typename T>
-__global__ void __launch_bounds__(NT) decode_combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
   extern __shared__ float sm[];
-  const int hq = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int hd = a.hd, H = a.H, Hq = a.Hkv * a.G, S = a.n_split, W = 2 * hd + H;
-  const int h = hq / a.G;
-  float* wsplit = sm;          // [S]
-  float* accs = wsplit + S;    // [W]
-  float* red = accs + W;       // [NT / 32]
-  const float* part = a.partials + ((size_t)b * Hq + hq) * S * a.part_stride;
-  float m = -CUDART_INF_F;
-  for (int s = tid; s < S; s += NT) m = fmaxf(m, part[(size_t)s * a.part_stride]);
-  m = warp_max(m);
-  if ((tid & 31) == 0) red[tid >> 5] = m;
-  __syncthreads();
-  float M = -CUDART_INF_F;
-  for (int i = 0; i < NT / 32; ++i) M = fmaxf(M, red[i]);
-  T* o = (T*)a.o + ((size_t)b * Hq + hq) * hd;
-  if (M == -CUDART_INF_F) {  // nothing attended: the output is zero
-    for (int j = tid; j < hd; j += NT) o[j] = from_f32<T>(0.f);
-    return;
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hd = a.hd, H = a.H, G = a.G, Hq = a.Hkv * a.G, S = a.n_split, W = 2 * hd + H;
+  float* wsplit = sm;              // [G][S]
+  float* accs = wsplit + G * S;    // [G][W]
+  float* inv_l = accs + G * W;     // [G]
+  float* mx = inv_l + G;           // [G]
+  const float* part0 = a.partials + ((size_t)b * Hq + (size_t)h * G) * S * a.part_stride;
+  // split maxima and weights, one warp per query head
+  for (int g = warp; g < G; g += CT / 32) {
+    const float* part = part0 + (size_t)g * S * a.part_stride;
+    float m = -CUDART_INF_F;
+    for (int s = lane; s < S; s += 32) m = fmaxf(m, part[(size_t)s * a.part_stride]);
+    m = warp_max(m);
+    float l = 0.f;
+    for (int s = lane; s < S; s += 32) {
+      const float ms = part[(size_t)s * a.part_stride];
+      const float wgt = (m == -CUDART_INF_F || ms == -CUDART_INF_F) ? 0.f : __expf(ms - m);
+      wsplit[g * S + s] = wgt;
+      l = fmaf(wgt, part[(size_t)s * a.part_stride + 1], l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) {
+      mx[g] = m;
+      inv_l[g] = l > 0.f ? 1.f / l : 0.f;
+    }
   }
-  for (int s = tid; s < S; s += NT) {
-    const float ms = part[(size_t)s * a.part_stride];
-    wsplit[s] = ms == -CUDART_INF_F ? 0.f : __expf(ms - M);
-  }
   __syncthreads();
-  float l = 0.f;
-  for (int s = 0; s < S; ++s) l = fmaf(wsplit[s], part[(size_t)s * a.part_stride + 1], l);
-  for (int e = tid; e < W; e += NT) {
+  for (int x = tid; x < G * W; x += CT) {
+    const int g = x / W, e = x % W;
+    const float* part = part0 + (size_t)g * S * a.part_stride + 4 + e;
+    const float* wg = wsplit + g * S;
     float v = 0.f;
-    for (int s = 0; s < S; ++s) v = fmaf(wsplit[s], part[(size_t)s * a.part_stride + 4 + e], v);
-    accs[e] = v;
+    for (int s = 0; s < S; ++s) v = fmaf(wg[s], part[(size_t)s * a.part_stride], v);
+    accs[x] = v;
   }
   __syncthreads();
   const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, h);
-  const float inv_l = 1.f / l;
-  for (int j = tid; j < hd; j += NT) {
-    float y = 0.f;
+  T* o = (T*)a.o + ((size_t)b * Hq + (size_t)h * G) * hd;
+  for (int j = warp; j < hd; j += CT / 32) {
     const T* wl = P.W_lin + (size_t)j * hd;
-    for (int i = 0; i < hd; ++i) y = fmaf(accs[i], to_f32(wl[i]), y);
     const T* w2 = P.W2 + (size_t)j * H;
-    for (int c = 0; c < H; ++c) y = fmaf(accs[hd + c], to_f32(w2[c]), y);
-    y = (y + accs[hd + H + j]) * inv_l;
-    if (P.b2) y += to_f32(P.b2[j]);
-    o[j] = from_f32<T>(y);
+    float wlv[8], w2v[16];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) wlv[q] = lane + 32 * q < hd ? to_f32(wl[lane + 32 * q]) : 0.f;
+#pragma unroll
+    for (int q = 0; q < 16; ++q) w2v[q] = lane + 32 * q < H ? to_f32(w2[lane + 32 * q]) : 0.f;
+    const float bj = P.b2 ? to_f32(P.b2[j]) : 0.f;
+    for (int g = 0; g < G; ++g) {
+      const float* ac = accs + g * W;
+      float y = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (lane + 32 * q < hd) y = fmaf(ac[lane + 32 * q], wlv[q], y);
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (lane + 32 * q < H) y = fmaf(ac[hd + lane + 32 * q], w2v[q], y);
+      y = warp_sum(y);
+      if (lane == 0) {
+        const float out = mx[g] == -CUDART_INF_F ? 0.f : (y + ac[hd + H + j]) * inv_l[g] + bj;
+        o[(size_t)g * hd + j] = from_f32<T>(out);
+      }
+    }
   }
 }
 
@@ -216,8 +240,8 @@ size_t decode_general_smem_bytes(int hd, int H, int G) {
   return (size_t)decode_smem_plan(hd, H, G).total * sizeof(float);
 }
 
-size_t decode_combine_smem_bytes(int hd, int H, int n_split) {
-  return (size_t)(n_split + 2 * hd + H + NT / 32) * sizeof(float);
+size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split) {
+  return (size_t)(G * n_split + G * (2 * hd + H) + 2 * G) * sizeof(float);
 }
 
 cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
@@ -237,17 +261,17 @@ cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
-  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.n_split);
-  dim3 grid(a.Hkv * a.G, a.B);
+  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.G, a.n_split);
+  dim3 grid(a.Hkv, a.B);
   cudaError_t e;
   if (dt == LR_BF16) {
     e = cudaFuncSetAttribute(decode_combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(a);
+    decode_combine_kernel<__nv_bfloat16><<<grid, CT, smem, st>>>(a);
   } else {
     e = cudaFuncSetAttribute(decode_combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<float><<<grid, NT, smem, st>>>(a);
+    decode_combine_kernel<float><<<grid, CT, smem, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -1,26 +1,29 @@
-// Tensor-core decode over the compressed cache (bf16, head_dim 128, sm_100a).
+// Tensor-core decode over the compressed cache (bf16 cache, head_dim 128, sm_100a).
 //
 // One CTA owns (split, KV-head pair, sequence) and walks 128-token tiles (two
 // 64-token blocks: consecutive blocks in full mode, entries of the pair's
 // selected-block union in selective mode). Per tile:
-//   MMA1  S1[128 x 256]  = A_tile[128 x r] . [B_l^a | B_l^b]^T   (keys of both heads:
-//                          "LowRAM" project page, Figure 3)
-//   epilogue  scores q.k~ in fp32 from TMEM, k~ -> fp16 tile in shared memory,
-//             online softmax -> p (fp16 tile)
-//   MMA2  U[128 x 128]   = k~ . W1_half^T          (GELU branch input, per 128 hidden)
-//   epilogue  g = GELU(U + b1) -> fp16 tile         ("Predicting the value cache from
-//                                                     keys", paragraphs 2-3)
-//   MMA3  O3 += g^T . p, k~^T . p                   (p-weighted sums, fp32 in TMEM)
+//   MMA1  S1[128 x 256] = A_tile[128 x r] . [B_l^a | B_l^b]^T   keys of both heads
+//                                            ("LowRAM" project page, Figure 3)
+//         SC[128 x 4G]  = A_tile . Qhat^T    scores q.k~ = A . (B_l^h q) for both heads,
+//                                            Qhat split into bf16 hi + lo rows
+//   epilogue  k~ -> fp16 tile in shared memory; online softmax -> p (fp16 tile)
+//   MMA2  U[128 x 128]  = k~ . W1_half^T     GELU-branch input, per 128 hidden units
+//   epilogue  g = GELU(U + b1) -> fp16 tile  ("Predicting the value cache from keys",
+//                                            paragraphs 2-3)
+//   MMA3  O3 = g^T . p, k~^T . p             p-weighted sums per dim, fp32 in TMEM
 //   epilogue  merge O3 into register accumulators with the softmax rescale and add
-//             p r over the tile's residual rows     (paragraph 2)
+//             p r over the tile's residual rows (paragraph 2)
 // The second-stage operands (k~, g, p and W1) are fp16: 11 significant bits keep the
 // rebuilt values within the attention tolerance even when one token dominates.
-// Roles: warp 0 issues TMA loads into a 3-stage ring (A and B_l chunks of 64 rank
-// columns, then W1 halves), warp 1 issues the MMAs, warps 2-5 run the epilogue.
-// The split partials (m, l, sum p k~, sum p g, sum p r) go to the same combine
-// kernel as the general path. Every wait is bounded: on a timeout the CTA records
-// LR_DEVERR_TIMEOUT, drains what it issued and returns.
+// Roles: warp 0 issues TMA loads into a 3-stage ring (A, B_l and Qhat chunks of 64
+// rank columns, then W1 halves), warp 1 issues the MMAs, warps 2-5 run the epilogue.
+// A prep kernel converts the layer's W1 to fp16, forms Qhat and (selective mode)
+// merges each pair's block lists. The split partials (m, l, sum p k~, sum p g,
+// sum p r) go to the same combine kernel as the general path. Every wait is bounded:
+// on a timeout the CTA records LR_DEVERR_TIMEOUT, drains what it issued and returns.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <math_constants.h>
 
 #include "lr_common.cuh"
@@ -35,46 +38,64 @@ namespace {
 using namespace sm100;
 
 constexpr int kHd = 128;
-constexpr int kChunk = 64;                 // rank columns per ring stage
+constexpr int kChunk = 64;  // rank columns per ring stage
 constexpr int kStages = 3;
-constexpr uint32_t kStageBytes = 48 * 1024;  // A rows 2 x 8 KB + B_l rows 2 x 16 KB
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6 residual rows
 constexpr int kEpi = 128;
 
 constexpr uint32_t kColS1 = 0;
 constexpr uint32_t kColU = 256;
 constexpr uint32_t kColO3 = 384;
+constexpr uint32_t kColSC = 480;
 constexpr uint32_t kTmemCols = 512;
 
-constexpr uint32_t kOffRing = 0;
-constexpr uint32_t kOffKt = kStages * kStageBytes;
-constexpr uint32_t kOffG = kOffKt + 32768;
-constexpr uint32_t kOffP = kOffG + 32768;
-constexpr uint32_t kOffQ = kOffP + 4096;
-constexpr uint32_t kOffB1 = kOffQ + 8192;
-constexpr uint32_t kOffRed = kOffB1 + 2048;
-constexpr uint32_t kOffBar = kOffRed + 256;
-constexpr uint32_t kOffMisc = kOffBar + 256;
-constexpr uint32_t kSmemUsed = kOffMisc + 64;
-constexpr uint32_t kSmemBytes = kSmemUsed + 1024;  // slack to align the base to 1024
+template <int MG>
+struct Layout {
+  static constexpr uint32_t kQRows = 4 * MG;                      // Qhat rows: 2 heads x (hi, lo) x MG
+  static constexpr uint32_t kQBytes = kQRows * 128;               // one 64-column chunk of Qhat
+  static constexpr uint32_t kStageBytes = 49152 + kQBytes;        // A 16 KB, B_l 32 KB, Qhat
+  static constexpr uint32_t kStageTx = kStageBytes;
+  static constexpr uint32_t kOffRing = 0;
+  static constexpr uint32_t kOffKt = (kStages * kStageBytes + 1023) & ~1023u;
+  static constexpr uint32_t kOffG = kOffKt + 32768;
+  static constexpr uint32_t kOffP = kOffG + 32768;
+  static constexpr uint32_t kOffB1 = kOffP + 4096;    // fp16 b1 of both heads (1 KB)
+  static constexpr uint32_t kOffRed = kOffB1 + 1024;  // 4 warps x 16 floats
+  static constexpr uint32_t kOffBar = kOffRed + 256;
+  static constexpr uint32_t kOffMisc = kOffBar + 256;
+  static constexpr uint32_t kOffAlpha = kOffMisc + 16;  // softmax rescale per (head slot, query head)
+  static constexpr uint32_t kSmemBytes = kOffMisc + 128 + 1024;  // + alignment slack
+};
+static_assert(Layout<8>::kSmemBytes <= 232448, "shared memory budget");
 
 enum Bar {
   FULL0 = 0, EMPTY0 = kStages, S1_FULL = 2 * kStages, S1_FREE, KT_READY, KT_FREE, U_FULL, U_FREE,
-  G_READY, G_FREE, O3_FULL0, O3_FULL1, O3_FREE0, O3_FREE1, DRAIN, EPI_SYNC, N_BARS
+  G_READY, G_FREE, O3_FULL0, O3_FULL1, O3_FREE0, O3_FREE1, DRAIN, EPI_SYNC, RES_READY, RES_DONE, N_BARS
 };
 static_assert(N_BARS * 8 <= 256, "barrier area");
 
-// GELU(x) = x Phi(x) with Phi(x) ~ (1 + tanh(x (c1 + c3 x^2 + c5 x^4 + c7 x^6))) / 2, x
-// clamped to [-6, 6] inside tanh. Coefficients are a minimax fit to the exact erf form
-// (max abs error 1.2e-5 in exact arithmetic; csrc/gelu_fit.py reproduces them).
-constexpr float kG1 = 7.97690120e-01f, kG3 = 3.67308140e-02f, kG5 = -2.55099297e-04f, kG7 = -8.60763669e-06f;
+// GELU(x) = x Phi(x) with Phi(x) ~ (1 + tanh(x (c1 + c3 x^2))) / 2, evaluated on two fp16
+// values at once. c1, c3 are a minimax fit to the exact erf form rounded to fp16 (max abs
+// error 3.0e-4 in exact arithmetic; csrc/gelu_fit.py reproduces them).
+constexpr uint32_t kGeluC1x2 = 0x3A673A67u;   // 0.80029297
+constexpr uint32_t kGeluC3x2 = 0x28712871u;   // 0.03469849
+constexpr uint32_t kHalfx2 = 0x38003800u;     // 0.5
 
-__device__ __forceinline__ float gelu_tc(float x) {
-  const float c = fminf(fmaxf(x, -6.f), 6.f);
-  const float s = c * c;
-  const float z = c * fmaf(s, fmaf(s, fmaf(s, kG7, kG5), kG3), kG1);
-  const float h = 0.5f * x;
-  return fmaf(h, tanh_fast(z), h);
+__device__ __forceinline__ uint32_t gelu_f16x2(uint32_t x) {
+  uint32_t s, p, z, t, h, g;
+  asm("mul.rn.f16x2 %0, %1, %1;" : "=r"(s) : "r"(x));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(p) : "r"(s), "r"(kGeluC3x2), "r"(kGeluC1x2));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(z) : "r"(x), "r"(p));
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(z));
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(h) : "r"(x), "r"(kHalfx2));
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(g) : "r"(h), "r"(t), "r"(h));
+  return g;
+}
+
+__device__ __forceinline__ uint32_t add_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -140,12 +161,12 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t atom_by
 
 template <int MG>
 struct HeadState {
-  float m[MG], l[MG], ak[MG], ag0[MG], ag1[MG], ar[MG];
+  float m[MG], l[MG], ak[MG], ag0[MG], ag1[MG];
   __device__ __forceinline__ void init() {
 #pragma unroll
     for (int g = 0; g < MG; ++g) {
       m[g] = -CUDART_INF_F;
-      l[g] = ak[g] = ag0[g] = ag1[g] = ar[g] = 0.f;
+      l[g] = ak[g] = ag0[g] = ag1[g] = 0.f;
     }
   }
 };
@@ -179,51 +200,49 @@ __device__ __forceinline__ bool epi_sync(EpiCtx& c) {
 // The epilogue's work for one KV head (slot HX of the pair) on the current tile.
 template <int HX, int MG>
 __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<MG>& st) {
+  using L = Layout<MG>;
   const int G = a.G, nh = a.H / 128;
   uint64_t* bars = c.bars;
-  const float* qs = reinterpret_cast<const float*>(c.sm + kOffQ);
-  const float* b1s = reinterpret_cast<const float*>(c.sm + kOffB1);
-  float* red = reinterpret_cast<float*>(c.sm + kOffRed);
-  uint8_t* ktile = c.sm + kOffKt;
-  uint8_t* gtile = c.sm + kOffG;
-  uint8_t* ptile = c.sm + kOffP;
+  const uint4* b1h = reinterpret_cast<const uint4*>(c.sm + L::kOffB1 + HX * 512);
+  float* red = reinterpret_cast<float*>(c.sm + L::kOffRed);
+  uint8_t* ktile = c.sm + L::kOffKt;
+  uint8_t* gtile = c.sm + L::kOffG;
+  uint8_t* ptile = c.sm + L::kOffP;
   const int row = c.row, lane = c.lane;
   const int n_kt = 2 * c.tl + HX;
   if (n_kt > 0 && !ewait(&bars[KT_FREE], (n_kt - 1) & 1, c.abort_flag)) return false;
-  // ---- scores and the fp16 key tile
+  // ---- scores (hi + lo columns) and the fp16 key tile
   float sc[MG];
+  {
+    uint32_t sv[2 * MG];
+    if constexpr (MG == 4) {
+      uint32_t t8[8];
+      tmem_ld8(c.trow + kColSC + HX * 8, t8);
 #pragma unroll
-  for (int g = 0; g < MG; ++g) sc[g] = 0.f;
+      for (int i = 0; i < 8; ++i) sv[i] = t8[i];
+    } else {
+      uint32_t t32[32];
+      tmem_ld32(c.trow + kColSC, t32);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sv[i] = t32[HX * 16 + i];
+    }
 #pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {
-    uint32_t v[32];
-    tmem_ld32(c.trow + kColS1 + HX * 128 + cc * 32, v);
-    tmem_ld_wait();
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t v[32];
+      tmem_ld32(c.trow + kColS1 + HX * 128 + cc * 32, v);
+      tmem_ld_wait();
 #pragma unroll
-    for (int g = 0; g < MG; ++g) {
-      if (g < G) {
-        const float4* q4 = reinterpret_cast<const float4*>(qs + (HX * 8 + g) * kHd + cc * 32);
-        float acc = sc[g];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 qq = q4[j];
-          acc = fmaf(__uint_as_float(v[4 * j]), qq.x, acc);
-          acc = fmaf(__uint_as_float(v[4 * j + 1]), qq.y, acc);
-          acc = fmaf(__uint_as_float(v[4 * j + 2]), qq.z, acc);
-          acc = fmaf(__uint_as_float(v[4 * j + 3]), qq.w, acc);
-        }
-        sc[g] = acc;
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_f16x2_sat(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
+        w.y = pack_f16x2_sat(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
+        w.z = pack_f16x2_sat(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
+        w.w = pack_f16x2_sat(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
+        *reinterpret_cast<uint4*>(ktile + sw128_off(row, cc * 32 + q * 8, 16384)) = w;
       }
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint4 w;
-      w.x = pack_f16x2_sat(__uint_as_float(v[8 * q + 0]), __uint_as_float(v[8 * q + 1]));
-      w.y = pack_f16x2_sat(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
-      w.z = pack_f16x2_sat(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
-      w.w = pack_f16x2_sat(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-      *reinterpret_cast<uint4*>(ktile + sw128_off(row, cc * 32 + q * 8, 16384)) = w;
-    }
+    for (int g = 0; g < MG; ++g) sc[g] = __uint_as_float(sv[g]) + __uint_as_float(sv[MG + g]);
   }
   if (HX == 1) {
     tc_fence_before();
@@ -248,12 +267,20 @@ __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<M
     st.l[g] = st.l[g] * alpha[g] + p[g];
     st.m[g] = m_new;
   }
+  // the residual warp has finished with the previous head's p tile
+  if (n_kt > 0 && !ewait(&bars[RES_DONE], (n_kt - 1) & 1, c.abort_flag)) return false;
 #pragma unroll
   for (int g = 0; g < MG; ++g)
     if (g < G) *reinterpret_cast<__half*>(ptile + sw128_off(g, row, 2048)) = __float2half_rn(p[g]);
+  if (row == 0) {
+    float* al = reinterpret_cast<float*>(c.sm + L::kOffAlpha) + HX * 8;
+#pragma unroll
+    for (int g = 0; g < MG; ++g) al[g] = alpha[g];
+  }
   fence_proxy_async_smem();
-  if (!epi_sync(c)) return false;  // p tile complete (read back below) and red consumed
+  if (!epi_sync(c)) return false;  // p tile and alpha complete; red consumed
   mbar_arrive(&bars[KT_READY]);
+  if (row == 0) mbar_arrive(&bars[RES_READY]);
   // ---- GELU branch, one 128-unit half at a time
 #pragma unroll 1
   for (int half = 0; half < nh; ++half) {
@@ -267,17 +294,16 @@ __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<M
     tc_fence_before();
     mbar_arrive(&bars[U_FREE]);
     if (j > 0 && !ewait(&bars[G_FREE], (j - 1) & 1, c.abort_flag)) return false;
-    const float* bb = b1s + HX * 256 + half * 128;
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
-      const int col = q * 8;
       const uint32_t* uu = &u[q >> 2][(q & 3) * 8];
+      const uint4 bb = b1h[half * 16 + q];
       uint4 w;
-      w.x = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[0]) + bb[col + 0]), gelu_tc(__uint_as_float(uu[1]) + bb[col + 1]));
-      w.y = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[2]) + bb[col + 2]), gelu_tc(__uint_as_float(uu[3]) + bb[col + 3]));
-      w.z = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[4]) + bb[col + 4]), gelu_tc(__uint_as_float(uu[5]) + bb[col + 5]));
-      w.w = pack_f16x2_sat(gelu_tc(__uint_as_float(uu[6]) + bb[col + 6]), gelu_tc(__uint_as_float(uu[7]) + bb[col + 7]));
-      *reinterpret_cast<uint4*>(gtile + sw128_off(row, col, 16384)) = w;
+      w.x = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[0]), __uint_as_float(uu[1])), bb.x));
+      w.y = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[2]), __uint_as_float(uu[3])), bb.y));
+      w.z = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[4]), __uint_as_float(uu[5])), bb.z));
+      w.w = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[6]), __uint_as_float(uu[7])), bb.w));
+      *reinterpret_cast<uint4*>(gtile + sw128_off(row, q * 8, 16384)) = w;
     }
     fence_proxy_async_smem();
     mbar_arrive(&bars[G_READY]);
@@ -297,50 +323,6 @@ __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<M
     st.ak[g] = fmaf(st.ak[g], alpha[g], __uint_as_float(ok8[g]));
     st.ag0[g] = fmaf(st.ag0[g], alpha[g], __uint_as_float(og0[g]));
     st.ag1[g] = fmaf(st.ag1[g], alpha[g], __uint_as_float(og1[g]));
-    st.ar[g] *= alpha[g];
-  }
-  // ---- residual rows of the tile's blocks: ar += p_t r_t[dim]
-  if (a.k > 0) {
-    const size_t seg = c.pseg + HX;
-    const int* ridx = a.res_idx + seg * a.k;
-    const __nv_bfloat16* rval = a.res_val + seg * a.k * kHd;
-    const int* rptr = a.res_ptr ? a.res_ptr + seg * (a.nblk + 1) : nullptr;
-#pragma unroll 1
-    for (int bh = 0; bh < 2; ++bh) {
-      const int blk = c.t.blk[bh];
-      if (blk < 0 || !((c.t.mask[bh] >> HX) & 1)) continue;
-      int e0, e1;
-      if (rptr) {
-        e0 = rptr[blk];
-        e1 = rptr[blk + 1];
-        if (e0 < 0 || e1 < e0 || e1 > a.k) {
-          if (row == 0) flag_error(a.err, LR_DEVERR_PTR);
-          continue;
-        }
-      } else {
-        e0 = lower_bound_i32(ridx, a.k, blk * kBlock);
-        e1 = lower_bound_i32(ridx, a.k, blk * kBlock + kBlock);
-      }
-      const int lo = blk * kBlock, hi = min(lo + kBlock, a.T);
-#pragma unroll 1
-      for (int e = e0; e < e1; ++e) {
-        const int tr = ridx[e];
-        if (tr < lo || tr >= hi) {
-          if (row == 0) flag_error(a.err, LR_DEVERR_RES_RANGE);
-          continue;
-        }
-        if (e > e0 && ridx[e - 1] >= tr && row == 0) flag_error(a.err, LR_DEVERR_RES_ORDER);
-        const float rv = __bfloat162float(rval[(size_t)e * kHd + row]);
-        const int prow = bh * 64 + (tr - lo);
-#pragma unroll
-        for (int g = 0; g < MG; ++g) {
-          if (g < G) {
-            const float pg = __half2float(*reinterpret_cast<const __half*>(ptile + sw128_off(g, prow, 2048)));
-            st.ar[g] = fmaf(pg, rv, st.ar[g]);
-          }
-        }
-      }
-    }
   }
   return true;
 }
@@ -348,7 +330,8 @@ __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<M
 template <int MG>
 __device__ __forceinline__ void write_partials(const TcArgs& a, EpiCtx& c, const HeadState<MG>& s0,
                                                const HeadState<MG>& s1, int b, int split, int ha) {
-  float* red = reinterpret_cast<float*>(c.sm + kOffRed);
+  using L = Layout<MG>;
+  float* red = reinterpret_cast<float*>(c.sm + L::kOffRed);
   epi_sync(c);  // red is free
 #pragma unroll
   for (int g = 0; g < MG; ++g) {
@@ -377,7 +360,139 @@ __device__ __forceinline__ void write_partials(const TcArgs& a, EpiCtx& c, const
       part[4 + row] = st.ak[g];
       part[4 + kHd + row] = st.ag0[g];
       if (a.H == 256) part[4 + kHd + 128 + row] = st.ag1[g];
-      part[4 + kHd + a.H + row] = st.ar[g];
+    }
+  }
+}
+
+// The residual warp: for each (tile, head) it scatters p_t r_t over the residual rows of the
+// tile's blocks ("Predicting the value cache from keys", paragraph 2). Lane l owns dims
+// 4l .. 4l+3; the rows of a block are contiguous in res_val (indices ascending), so a batch
+// of 16 rows is one coalesced 256-byte read per row. Loads are issued before waiting for
+// the epilogue's p tile, so their latency overlaps the softmax.
+template <int MG>
+__device__ __forceinline__ void residual_warp(const TcArgs& a, uint8_t* sm, uint64_t* bars, volatile int* abort_flag,
+                                              int b, int hp, int split, int t_begin, int t_end) {
+  using L = Layout<MG>;
+  const int lane = threadIdx.x & 31, ha = 2 * hp, G = a.G;
+  const uint8_t* ptile = sm + L::kOffP;
+  const float* alphas = reinterpret_cast<const float*>(sm + L::kOffAlpha);
+  float acc[2][MG][4];
+#pragma unroll
+  for (int hx = 0; hx < 2; ++hx)
+#pragma unroll
+    for (int g = 0; g < MG; ++g)
+#pragma unroll
+      for (int d = 0; d < 4; ++d) acc[hx][g][d] = 0.f;
+  int bad = 0;
+  bool ok = true;
+  int tl = 0;
+  const size_t pseg = ((size_t)b * a.L + a.layer) * a.Hkv + ha;
+  for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
+    const TileInfo t = tile_info(a, b, hp, ti);
+#pragma unroll
+    for (int hx = 0; hx < 2; ++hx) {
+      if (!ok) break;
+      const int n_kt = 2 * tl + hx;
+      int e0[2] = {0, 0}, ne[2] = {0, 0}, lo[2] = {0, 0}, hi[2] = {0, 0};
+      const int* ridx = nullptr;
+      const __nv_bfloat16* rval = nullptr;
+      if (a.k > 0) {
+        const size_t seg = pseg + hx;
+        ridx = a.res_idx + seg * a.k;
+        rval = a.res_val + seg * a.k * kHd;
+        const int* rptr = a.res_ptr ? a.res_ptr + seg * (a.nblk + 1) : nullptr;
+#pragma unroll
+        for (int bh = 0; bh < 2; ++bh) {
+          const int blk = t.blk[bh];
+          if (blk < 0 || !((t.mask[bh] >> hx) & 1)) continue;
+          int x0, x1;
+          if (rptr) {
+            x0 = __ldg(rptr + blk);
+            x1 = __ldg(rptr + blk + 1);
+            if (x0 < 0 || x1 < x0 || x1 > a.k) {
+              bad |= LR_DEVERR_PTR;
+              continue;
+            }
+          } else {
+            x0 = lower_bound_i32(ridx, a.k, blk * kBlock);
+            x1 = lower_bound_i32(ridx, a.k, blk * kBlock + kBlock);
+          }
+          e0[bh] = x0;
+          ne[bh] = x1 - x0;
+          lo[bh] = blk * kBlock;
+          hi[bh] = min(lo[bh] + kBlock, a.T);
+        }
+      }
+      const int n_tot = ne[0] + ne[1];
+      bool waited = false;
+#pragma unroll 1
+      for (int i0 = 0; i0 < n_tot || !waited; i0 += 16) {
+        int tr[16], bh_of[16];
+        uint2 rv[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int i = i0 + j;
+          const int bh = i < ne[0] ? 0 : 1;
+          const int e = bh ? e0[1] + (i - ne[0]) : e0[0] + i;
+          const bool in = i < n_tot;
+          bh_of[j] = bh;
+          tr[j] = in ? __ldg(ridx + e) : -1;
+          rv[j] = in ? __ldg(reinterpret_cast<const uint2*>(rval + (size_t)e * kHd) + lane) : make_uint2(0, 0);
+        }
+        if (!waited) {
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&bars[RES_READY], n_kt & 1, abort_flag)))) break;
+          waited = true;
+#pragma unroll
+          for (int g = 0; g < MG; ++g) {
+            const float al = alphas[hx * 8 + g];
+#pragma unroll
+            for (int d = 0; d < 4; ++d) acc[hx][g][d] *= al;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          if (i0 + j >= n_tot) break;
+          const int bh = bh_of[j];
+          if (j > 0 && bh_of[j - 1] == bh && tr[j - 1] >= tr[j]) bad |= LR_DEVERR_RES_ORDER;
+          if (tr[j] < lo[bh] || tr[j] >= hi[bh]) {
+            bad |= LR_DEVERR_RES_RANGE;
+            continue;
+          }
+          const int prow = bh * 64 + (tr[j] - lo[bh]);
+          const __nv_bfloat162 r01 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].x);
+          const __nv_bfloat162 r23 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].y);
+          const float r0 = __low2float(r01), r1 = __high2float(r01), r2 = __low2float(r23), r3 = __high2float(r23);
+#pragma unroll
+          for (int g = 0; g < MG; ++g) {
+            if (g < G) {
+              const float pg = __half2float(*reinterpret_cast<const __half*>(ptile + sw128_off(g, prow, 2048)));
+              acc[hx][g][0] = fmaf(pg, r0, acc[hx][g][0]);
+              acc[hx][g][1] = fmaf(pg, r1, acc[hx][g][1]);
+              acc[hx][g][2] = fmaf(pg, r2, acc[hx][g][2]);
+              acc[hx][g][3] = fmaf(pg, r3, acc[hx][g][3]);
+            }
+          }
+        }
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[RES_DONE]);
+    }
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    flag_error(a.err, LR_DEVERR_TIMEOUT);
+  }
+  if (bad && lane == 0) flag_error(a.err, bad);
+  const int Hq = a.Hkv * G;
+#pragma unroll
+  for (int hx = 0; hx < 2; ++hx) {
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      if (g >= G) continue;
+      float* part = a.partials + (((size_t)b * Hq + (ha + hx) * G + g) * a.n_split + split) * a.part_stride;
+      *reinterpret_cast<float4*>(part + 4 + kHd + a.H + 4 * lane) =
+          make_float4(acc[hx][g][0], acc[hx][g][1], acc[hx][g][2], acc[hx][g][3]);
     }
   }
 }
@@ -385,16 +500,18 @@ __device__ __forceinline__ void write_partials(const TcArgs& a, EpiCtx& c, const
 template <int MG>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                 const __grid_constant__ CUtensorMap mapW1, const TcArgs a) {
+                 const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapW1,
+                 const TcArgs a) {
+  using L = Layout<MG>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kOffBar);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kOffMisc + 4);
 
   const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = a.G, H = a.H, nh = a.H / 128, nk = a.r / kChunk;
+  const int H = a.H, nh = a.H / 128, nk = a.r / kChunk;
   const int n_tiles = tile_count(a, b, hp);
   const int t_begin = (int)((long long)s * n_tiles / a.n_split);
   const int t_end = (int)((long long)(s + 1) * n_tiles / a.n_split);
@@ -420,32 +537,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     mbar_init(&bars[O3_FREE1], kEpi);
     mbar_init(&bars[DRAIN], 1);
     mbar_init(&bars[EPI_SYNC], kEpi);
+    mbar_init(&bars[RES_READY], 1);
+    mbar_init(&bars[RES_DONE], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapA);
     tma_prefetch_desc(&mapB);
+    tma_prefetch_desc(&mapQ);
     tma_prefetch_desc(&mapW1);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, kTmemCols);
     tmem_relinquish();
   }
-  {  // query rows of the pair (pre-scaled), b1 of both heads, zero p tile
-    float* qs = reinterpret_cast<float*>(sm + kOffQ);
-    const __nv_bfloat16* q = a.q + ((size_t)b * a.Hkv * G + (size_t)ha * G) * kHd;
-    for (int i = threadIdx.x; i < 2 * 8 * kHd; i += kThreads) {
-      const int hx = i / (8 * kHd), g = (i / kHd) % 8, d = i % kHd;
-      qs[i] = g < G ? __bfloat162float(q[((size_t)hx * G + g) * kHd + d]) * a.scale : 0.f;
-    }
-    float* b1s = reinterpret_cast<float*>(sm + kOffB1);
+  {  // b1 of both heads as fp16, zero p tile
+    __half* b1s = reinterpret_cast<__half*>(sm + L::kOffB1);
     const size_t pseq = a.pred_per_seq ? (size_t)b : 0;
     for (int i = threadIdx.x; i < 2 * 256; i += kThreads) {
       const int hx = i / 256, c = i % 256;
-      b1s[i] = c < H ? __bfloat162float(a.b1[((pseq * a.L + a.layer) * a.Hkv + ha + hx) * H + c]) : 0.f;
+      b1s[i] = __float2half_rn(
+          c < H ? __bfloat162float(a.b1[((pseq * a.L + a.layer) * a.Hkv + ha + hx) * H + c]) : 0.f);
     }
-    uint32_t* pz = reinterpret_cast<uint32_t*>(sm + kOffP);
+    uint32_t* pz = reinterpret_cast<uint32_t*>(sm + L::kOffP);
     for (int i = threadIdx.x; i < 1024; i += kThreads) pz[i] = 0u;
   }
   fence_proxy_async_smem();
@@ -460,6 +575,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       uint32_t it = 0;
       bool ok = true;
       const int rowB = (a.layer * a.Hkv + ha) * kHd;
+      const int rowQ = (b * a.n_hp + hp) * (int)L::kQRows;
       const int w1seq = a.pred_per_seq ? b : 0;
       for (int ti = t_begin; ti < t_end && ok; ++ti) {
         const TileInfo t = tile_info(a, b, hp, ti);
@@ -468,18 +584,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
         for (int kc = 0; kc < nk && ok; ++kc, ++it) {
           const uint32_t st = it % kStages, ph = (it / kStages) & 1;
           if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
-          uint8_t* dst = sm + kOffRing + st * kStageBytes;
-          mbar_arrive_expect_tx(&bars[FULL0 + st], kStageBytes);
+          uint8_t* dst = sm + L::kOffRing + st * L::kStageBytes;
+          mbar_arrive_expect_tx(&bars[FULL0 + st], L::kStageTx);
           tma_load_3d(dst, &mapA, &bars[FULL0 + st], kc * kChunk, row0, b);
           tma_load_3d(dst + 8192, &mapA, &bars[FULL0 + st], kc * kChunk, row1, b);
           tma_load_3d(dst + 16384, &mapB, &bars[FULL0 + st], kc * kChunk, rowB, b);
           tma_load_3d(dst + 32768, &mapB, &bars[FULL0 + st], kc * kChunk, rowB + kHd, b);
+          tma_load_2d(dst + 49152, &mapQ, &bars[FULL0 + st], kc * kChunk, rowQ);
         }
         for (int hx = 0; hx < 2 && ok; ++hx) {
           for (int half = 0; half < nh && ok; ++half, ++it) {
             const uint32_t st = it % kStages, ph = (it / kStages) & 1;
             if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
-            uint8_t* dst = sm + kOffRing + st * kStageBytes;
+            uint8_t* dst = sm + L::kOffRing + st * L::kStageBytes;
             const int wrow = ((w1seq * a.Hkv + ha + hx) * H) + half * 128;
             mbar_arrive_expect_tx(&bars[FULL0 + st], 32768);
             tma_load_2d(dst, &mapW1, &bars[FULL0 + st], 0, wrow);
@@ -499,9 +616,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_s1 = idesc_bf16_f32(128, 256, false, false);
+      const uint32_t id_sc = idesc_bf16_f32(128, L::kQRows, false, false);
       const uint32_t id_u = idesc_f16_f32(128, 128, false, false);
       const uint32_t id_o3 = idesc_f16_f32(128, 16, true, false);
-      const uint32_t kt = smem_u32(sm + kOffKt), gt = smem_u32(sm + kOffG), pt = smem_u32(sm + kOffP);
+      const uint32_t kt = smem_u32(sm + L::kOffKt), gt = smem_u32(sm + L::kOffG), pt = smem_u32(sm + L::kOffP);
       uint32_t it = 0;
       bool ok = true;
       int tl = 0;
@@ -512,11 +630,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
           const uint32_t st = it % kStages, ph = (it / kStages) & 1;
           if (!(ok = mbar_wait(&bars[FULL0 + st], ph, abort_flag))) break;
           tc_fence_after();
-          const uint32_t base = smem_u32(sm + kOffRing + st * kStageBytes);
+          const uint32_t base = smem_u32(sm + L::kOffRing + st * L::kStageBytes);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_f16_ss(tmem + kColS1, sw128_desc(base + ks * 32, 16, 1024),
-                        sw128_desc(base + 16384 + ks * 32, 16, 1024), id_s1, (kc | ks) != 0);
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t adesc = sw128_desc(base + ks * 32, 16, 1024);
+            mma_f16_ss(tmem + kColS1, adesc, sw128_desc(base + 16384 + ks * 32, 16, 1024), id_s1, (kc | ks) != 0);
+            mma_f16_ss(tmem + kColSC, adesc, sw128_desc(base + 49152 + ks * 32, 16, 1024), id_sc, (kc | ks) != 0);
+          }
           mma_commit(&bars[EMPTY0 + st]);
         }
         if (!ok) break;
@@ -532,12 +652,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
             if (!(ok = mbar_wait(&bars[FULL0 + st], ph, abort_flag))) break;
             if (!(ok = mbar_wait(&bars[U_FREE], (j & 1) ^ 1, abort_flag))) break;
             tc_fence_after();
-            const uint32_t wb = smem_u32(sm + kOffRing + st * kStageBytes);
+            const uint32_t wb = smem_u32(sm + L::kOffRing + st * L::kStageBytes);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
               const uint32_t off = (ks >> 2) * 16384 + (ks & 3) * 32;
               mma_f16_ss(tmem + kColU, sw128_desc(kt + off, 16, 1024), sw128_desc(wb + off, 16, 1024), id_u,
-                          ks != 0);
+                         ks != 0);
             }
             mma_commit(&bars[EMPTY0 + st]);
             mma_commit(&bars[U_FULL]);
@@ -549,14 +669,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
               mma_f16_ss(tmem + kColO3 + hx * 48 + 16 + half * 16, sw128_desc(gt + ks * 2048, 16384, 1024),
-                          sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
+                         sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
             mma_commit(&bars[G_FREE]);
           }
           if (!ok) break;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             mma_f16_ss(tmem + kColO3 + hx * 48, sw128_desc(kt + ks * 2048, 16384, 1024),
-                        sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
+                       sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
           mma_commit(&bars[KT_FREE]);
           mma_commit(&bars[O3_FULL0 + hx]);
         }
@@ -569,6 +689,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       mma_commit(&bars[DRAIN]);
       mbar_wait_drain(&bars[DRAIN], 0, kWaitCycles / 4);
     }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------------- residual rows
+    residual_warp<MG>(a, sm, bars, abort_flag, b, hp, s, t_begin, t_end);
   } else {
     // ---------------------------------------------------------------- epilogue
     EpiCtx c;
@@ -590,10 +713,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
       c.t = tile_info(a, b, hp, ti);
       const int half_row = c.row >> 6;
-      const int rblk = c.t.blk[half_row];
+      const int rblk = half_row ? c.t.blk[1] : c.t.blk[0];
       const int tok = rblk * kBlock + (c.row & 63);
       c.row_valid = rblk >= 0 && tok < a.T;
-      c.rmask = c.t.mask[half_row];
+      c.rmask = half_row ? c.t.mask[1] : c.t.mask[0];
       c.tl = tl;
       if (!(ok = ewait(&bars[S1_FULL], tl & 1, abort_flag))) break;
       tc_fence_after();
@@ -604,7 +727,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       *abort_flag = 1;
       flag_error(a.err, LR_DEVERR_TIMEOUT);
     }
-    write_partials(a, c, st0, st1, b, s, ha);
+    write_partials<MG>(a, c, st0, st1, b, s, ha);
   }
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
@@ -616,34 +739,75 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
   }
 }
 
-// The layer's W1 as fp16 (the second-stage MMAs take fp16 operands so that the rebuilt
-// keys and GELU outputs keep 11 significant bits). bf16 -> fp16 is exact except for
-// magnitudes below 2^-14 (fp16 subnormals) or above 65504 (saturated).
-__global__ void decode_tc_w1_kernel(TcArgs a) {
-  const size_t per_seq = (size_t)a.Hkv * a.H * kHd;
-  const size_t n = (size_t)a.w1_seqs * per_seq;
-  for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 4; i < n; i += (size_t)gridDim.x * blockDim.x * 4) {
-    const size_t sq = i / per_seq, r = i % per_seq;
-    const __nv_bfloat16* src = a.W1 + (sq * a.L + a.layer) * per_seq + r;
-    const uint2 v = *reinterpret_cast<const uint2*>(src);
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-    uint2 o;
-    o.x = pack_f16x2_sat(__low2float(lo), __high2float(lo));
-    o.y = pack_f16x2_sat(__low2float(hi), __high2float(hi));
-    *reinterpret_cast<uint2*>(a.W1h + i) = o;
+// Prep work of one decode call, one launch:
+//   blocks [0, n_w1)             the layer's W1 as fp16 (bf16 -> fp16 is exact except below
+//                                2^-14 or above 65504, where values saturate)
+//   blocks [n_w1, n_w1 + n_q)    Qhat = scale * B_l^h q for every query head, stored as bf16
+//                                hi + lo rows (hi = bf16(x), lo = bf16(x - hi)); one block per
+//                                (256 rank columns, KV head, sequence)
+//   blocks [n_w1 + n_q, ...)     selective mode: per (sequence, head pair) the union of the two
+//                                block lists with a 2-bit head mask (bit 0: first head); entries
+//                                out of range or not strictly ascending are skipped and flagged
+template <int MG>
+__global__ void __launch_bounds__(256) decode_tc_prep_kernel(TcArgs a, int n_w1, int n_q, const int* blocks,
+                                                             int n_sel) {
+  const int bid = blockIdx.x, tid = threadIdx.x;
+  if (bid < n_w1) {
+    const size_t per_seq = (size_t)a.Hkv * a.H * kHd;
+    const size_t n = (size_t)a.w1_seqs * per_seq;
+    for (size_t i = ((size_t)bid * 256 + tid) * 4; i < n; i += (size_t)n_w1 * 256 * 4) {
+      const size_t sq = i / per_seq, r = i % per_seq;
+      const uint2 v = *reinterpret_cast<const uint2*>(a.W1 + (sq * a.L + a.layer) * per_seq + r);
+      const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+      const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+      uint2 o;
+      o.x = pack_f16x2_sat(__low2float(lo), __high2float(lo));
+      o.y = pack_f16x2_sat(__low2float(hi), __high2float(hi));
+      *reinterpret_cast<uint2*>(a.W1h + i) = o;
+    }
+    return;
   }
-}
-
-// Per (sequence, KV-head pair): merge the two selected-block lists into one ascending
-// union with a 2-bit head mask per block (bit 0: first head, bit 1: second). Entries that
-// are out of range or not strictly ascending are skipped and flagged.
-__global__ void decode_tc_schedule_kernel(TcArgs a, const int* __restrict__ blocks, int n_sel, int* sched) {
-  const int hp = blockIdx.x, b = blockIdx.y;
-  if (threadIdx.x != 0) return;
+  if (bid < n_w1 + n_q) {
+    __shared__ float qs[8][kHd];
+    const int nj = (a.r + 255) / 256;
+    const int q = bid - n_w1;
+    const int jc = q % nj, h = (q / nj) % a.Hkv, b = q / (nj * a.Hkv);
+    const int G = a.G;
+    for (int i = tid; i < 8 * kHd; i += 256) {
+      const int g = i / kHd, d = i % kHd;
+      qs[g][d] = g < G ? __bfloat162float(a.q[(((size_t)b * a.Hkv + h) * G + g) * kHd + d]) * a.scale : 0.f;
+    }
+    __syncthreads();
+    const int j = jc * 256 + tid;
+    if (j >= a.r) return;
+    const size_t D = (size_t)a.L * a.Hkv * kHd;
+    const __nv_bfloat16* bt = a.Bt + (size_t)b * D * a.r + ((size_t)(a.layer * a.Hkv + h) * kHd) * a.r + j;
+    float acc[MG];
+#pragma unroll
+    for (int g = 0; g < MG; ++g) acc[g] = 0.f;
+#pragma unroll 4
+    for (int d = 0; d < kHd; ++d) {
+      const float v = __bfloat162float(bt[(size_t)d * a.r]);
+#pragma unroll
+      for (int g = 0; g < MG; ++g) acc[g] = fmaf(v, qs[g][d], acc[g]);
+    }
+    const int hp = h >> 1, hx = h & 1;
+    __nv_bfloat16* out = a.qhat + ((size_t)(b * a.n_hp + hp) * (4 * MG) + hx * 2 * MG) * a.r + j;
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(acc[g]);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(acc[g] - __bfloat162float(hi));
+      out[(size_t)g * a.r] = hi;
+      out[(size_t)(MG + g) * a.r] = lo;
+    }
+    return;
+  }
+  if (tid != 0) return;
+  const int q = bid - n_w1 - n_q;
+  const int hp = q % a.n_hp, b = q / a.n_hp;
   const int* la = blocks + ((size_t)b * a.Hkv + 2 * hp) * n_sel;
   const int* lb = la + n_sel;
-  int* out = sched + ((size_t)b * a.n_hp + hp) * a.sched_stride;
+  int* out = const_cast<int*>(a.sched) + ((size_t)b * a.n_hp + hp) * a.sched_stride;
   int i = 0, j = 0, n = 0, prev_a = -1, prev_b = -1, bits = 0;
   auto next = [&](const int* l, int& k, int& prev) -> int {
     while (k < n_sel) {
@@ -671,34 +835,31 @@ __global__ void decode_tc_schedule_kernel(TcArgs a, const int* __restrict__ bloc
   if (bits) flag_error(a.err, bits);
 }
 
+template <int MG>
+cudaError_t launch_mg(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mQ,
+                      const CUtensorMap& mW1, const int* blocks, int n_sel, cudaStream_t st) {
+  const size_t n_w1_vec = (size_t)a.w1_seqs * a.Hkv * a.H * kHd / 4;
+  const int n_w1 = (int)((n_w1_vec + 255) / 256 < 512 ? (n_w1_vec + 255) / 256 : 512);
+  const int n_q = ((a.r + 255) / 256) * a.Hkv * a.B;
+  const int n_s = a.sched ? a.n_hp * a.B : 0;
+  decode_tc_prep_kernel<MG><<<n_w1 + n_q + n_s, 256, 0, st>>>(a, n_w1, n_q, blocks, n_sel);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_tc_kernel<MG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)Layout<MG>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<MG><<<dim3(a.n_split, a.n_hp, a.B), kThreads, Layout<MG>::kSmemBytes, st>>>(mA, mB, mQ, mW1, a);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
-size_t decode_tc_smem_bytes() { return kSmemBytes; }
+int qhat_rows(int G) { return G <= 4 ? 16 : 32; }
 
-cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mW1,
-                             const int* blocks, int n_sel, cudaStream_t st) {
-  cudaError_t e;
-  {
-    const size_t n = (size_t)a.w1_seqs * a.Hkv * a.H * kHd / 4;
-    const int blocks_w1 = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-    decode_tc_w1_kernel<<<blocks_w1, 256, 0, st>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  if (a.sched) {
-    decode_tc_schedule_kernel<<<dim3(a.n_hp, a.B), 32, 0, st>>>(a, blocks, n_sel, const_cast<int*>(a.sched));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  const dim3 grid(a.n_split, a.n_hp, a.B);
-  if (a.G <= 4) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    decode_tc_kernel<4><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, mW1, a);
-  } else {
-    e = cudaFuncSetAttribute(decode_tc_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    decode_tc_kernel<8><<<grid, kThreads, kSmemBytes, st>>>(mA, mB, mW1, a);
-  }
-  return cudaGetLastError();
+cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mQ,
+                             const CUtensorMap& mW1, const int* blocks, int n_sel, cudaStream_t st) {
+  return a.G <= 4 ? launch_mg<4>(a, mA, mB, mQ, mW1, blocks, n_sel, st)
+                  : launch_mg<8>(a, mA, mB, mQ, mW1, blocks, n_sel, st);
 }
 
 }  // namespace tc

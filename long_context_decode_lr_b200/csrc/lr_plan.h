@@ -20,6 +20,7 @@ struct DecodePlan {
   size_t part_off;   // byte offset of the partials in the workspace
   size_t sched_off;  // byte offset of the tensor path's block schedule
   size_t w1h_off;    // byte offset of the tensor path's fp16 copy of the layer's W1
+  size_t qhat_off;   // byte offset of the tensor path's Qhat operand
   size_t ws_bytes;   // total workspace
 };
 

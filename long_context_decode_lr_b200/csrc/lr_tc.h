@@ -18,6 +18,8 @@ struct TcArgs {
   float scale;
   const __nv_bfloat16* q;        // [B, Hq, 128]
   const __nv_bfloat16* b1;       // [(B,) L, Hkv, H]
+  const __nv_bfloat16* Bt;       // [B, D, r]
+  __nv_bfloat16* qhat;           // workspace: [B, n_hp, 4*MG, r] scale * B_l^h q as bf16 hi/lo rows
   const __nv_bfloat16* W1;       // [(B,) L, Hkv, H, 128]
   __half* W1h;                   // workspace: [(B,) Hkv, H, 128] fp16 copy of the layer's W1
   int w1_seqs;                   // 1, or B when each sequence has its own predictor
@@ -31,9 +33,10 @@ struct TcArgs {
   int* err;
 };
 
-size_t decode_tc_smem_bytes();
-cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mW1,
-                             const int* blocks, int n_sel, cudaStream_t st);
+// Rows of the Qhat operand per (sequence, head pair): 2 heads x (hi, lo) x 4 or 8 query heads.
+int qhat_rows(int G);
+cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mQ,
+                             const CUtensorMap& mW1, const int* blocks, int n_sel, cudaStream_t st);
 
 }  // namespace tc
 }  // namespace lr

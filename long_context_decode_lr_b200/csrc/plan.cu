@@ -67,7 +67,9 @@ DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm
     const size_t sched_bytes = (size_t)rows * (1 + 2 * (size_t)(n_sel > 0 ? n_sel : 0)) * sizeof(int);
     p.w1h_off = align256(p.sched_off + sched_bytes);
     const size_t w1h_bytes = (size_t)s.batch * s.n_kv_heads * s.hidden * s.head_dim * 2;
-    p.ws_bytes = align256(p.w1h_off + w1h_bytes);
+    p.qhat_off = align256(p.w1h_off + w1h_bytes);
+    const size_t qhat_bytes = (size_t)rows * tc::qhat_rows(n_q_heads / s.n_kv_heads) * s.rank * 2;
+    p.ws_bytes = align256(p.qhat_off + qhat_bytes);
     return p;
   }
   p.path = DecodePath::General;
@@ -109,6 +111,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype 
     t.q = (const __nv_bfloat16*)a.q;
     t.b1 = (const __nv_bfloat16*)a.b1;
     t.W1 = (const __nv_bfloat16*)a.W1;
+    t.Bt = (const __nv_bfloat16*)a.Bt;
+    t.qhat = (__nv_bfloat16*)((char*)a.err + plan.qhat_off);
     t.W1h = (__half*)((char*)a.err + plan.w1h_off);
     t.w1_seqs = a.pred_per_seq ? a.B : 1;
     t.res_idx = a.res_idx;
@@ -120,7 +124,11 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype 
     t.part_stride = plan.part_stride;
     t.err = a.err;
     const cuuint64_t D = (cuuint64_t)a.L * a.Hkv * a.hd;
-    CUtensorMap mA, mB, mW1;
+    CUtensorMap mA, mB, mQ, mW1;
+    const cuuint64_t q_rows = (cuuint64_t)tc::qhat_rows(a.G);
+    const cuuint64_t dQ[2] = {(cuuint64_t)a.r, (cuuint64_t)a.B * t.n_hp * q_rows};
+    const cuuint64_t sQ[1] = {(cuuint64_t)a.r * 2};
+    const cuuint32_t bQ[2] = {64, (cuuint32_t)q_rows};
     const cuuint64_t dA[3] = {(cuuint64_t)a.r, (cuuint64_t)a.T, (cuuint64_t)a.B};
     const cuuint64_t sA[2] = {(cuuint64_t)a.r * 2, (cuuint64_t)a.T * a.r * 2};
     const cuuint32_t bA[3] = {64, 64, 1};
@@ -133,9 +141,10 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype 
     const cuuint32_t bW[2] = {64, 128};
     if (!tile_map(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, 3, dA, sA, bA) ||
         !tile_map(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Bt, 3, dB, sB, bB) ||
+        !tile_map(&mQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, t.qhat, 2, dQ, sQ, bQ) ||
         !tile_map(&mW1, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, t.W1h, 2, dW, sW, bW))
       return cudaErrorInvalidValue;
-    if ((e = tc::launch_decode_tc(t, mA, mB, mW1, a.blocks, a.n_sel, st)) != cudaSuccess) return e;
+    if ((e = tc::launch_decode_tc(t, mA, mB, mQ, mW1, a.blocks, a.n_sel, st)) != cudaSuccess) return e;
     return launch_decode_combine(a, dt, st);
   }
   e = launch_decode_general(a, dt, st);

@@ -179,6 +179,7 @@ def assert_attention_close(got, ref, rel_l2=REL_L2, max_abs=MAX_ABS):
     rel = np.linalg.norm(diff) / max(nref, 1e-30)
     mab = np.abs(diff).max() if diff.size else 0.0
     assert np.all(np.isfinite(got)), "non-finite output"
+    print(f"[attention parity] rel_l2={rel:.3e} max_abs={mab:.3e}")
     assert rel <= rel_l2 and mab <= max_abs, f"rel_l2={rel:.3e} max_abs={mab:.3e}"
     return rel, mab
 
