@@ -193,6 +193,39 @@ lr_status lr_topk_tokens(const float* err, int32_t n_segments, int32_t T, int32_
 lr_status lr_residual_block_ptr(const int32_t* idx, int32_t n_segments, int32_t k, int32_t T,
                                 int32_t* ptr_out, lr_stream_t stream);
 
+/* ------------------------------------------------------------------ allocation-free decode */
+
+/*
+ * lr_decode_attn_noalloc -- lr_decode_attn for callers that cannot allocate device memory.
+ * The paper has no counterpart: this is a deployment variant of the decode step above.
+ *
+ * Some callers cannot call cudaMalloc or any allocating routine: code running inside an
+ * allocator or memory-pool callback, runtimes that own every device allocation and only
+ * hand out fixed buffers, and latency-critical paths where an allocation could block or
+ * fail. This entry point takes the same inputs and output as lr_decode_attn (caller-owned
+ * device tensors) but no workspace: it runs on a 16 MiB scratch array compiled into the
+ * library (a file-scope __device__ array, present on every GPU that loads the library
+ * until the process exits).
+ *   - Shapes whose lr_decode_workspace_bytes exceeds 16 MiB return LR_ERR_WORKSPACE with
+ *     a message in lr_last_error(); nothing is launched.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array and each call clears the part that must start
+ *     at zero; calls that overlap on the GPU (different streams, or host threads without
+ *     ordering) race on it.
+ *   - Device-side data checks write the shared array's error word, which this entry point
+ *     does not expose; use lr_decode_attn with a workspace when you need
+ *     lr_get_device_error.
+ * Argument meaning, layouts, ownership and the other error behaviour: as lr_decode_attn.
+ */
+lr_status lr_decode_attn_noalloc(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
+                                 const void* q, const void* A, const void* Bt,
+                                 const lr_predictor* predictor, const int32_t* res_idx,
+                                 const void* res_val, const int32_t* res_blk_ptr, int32_t k,
+                                 const int32_t* block_list, int32_t n_sel, float scale, void* o,
+                                 lr_stream_t stream);
+
 /* ------------------------------------------------------------------ errors, version */
 
 /* Copies the device error word of the last call that used `ws` into *code and

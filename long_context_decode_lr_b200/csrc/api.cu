@@ -81,6 +81,11 @@ int current_sm_count() {
 
 }  // namespace
 
+namespace lr {
+// Records a message for lr_last_error() (used by entry points defined in other files).
+void set_last_error(const char* msg) { snprintf(g_msg, sizeof(g_msg), "%s", msg); }
+}  // namespace lr
+
 extern "C" {
 
 const char* lr_last_error(void) { return g_msg; }

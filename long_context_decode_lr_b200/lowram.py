@@ -62,6 +62,8 @@ def library() -> ctypes.CDLL:
             "lr_decode_workspace_bytes": (_Z, [S, _I, _I]),
             "lr_decode_attn": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _I, _P, _I, ctypes.c_float,
                                     _P, _P, _Z, _P]),
+            "lr_decode_attn_noalloc": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _I, _P, _I, ctypes.c_float,
+                                            _P, _P]),
             "lr_topk_workspace_bytes": (_Z, [_I, _I, _I]),
             "lr_topk_tokens": (_I, [_P, _I, _I, _I, _P, _P, _Z, _P]),
             "lr_residual_block_ptr": (_I, [_P, _I, _I, _I, _P, _P]),
@@ -141,6 +143,15 @@ def lr_decode_attn(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_
         ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
         _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, float(scale),
         _ptr(o), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def lr_decode_attn_noalloc(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_idx, res_val,
+                           res_blk_ptr, k, block_list, n_sel, scale, o, stream=None) -> None:
+    """lr_decode_attn on the library's static scratch area (no workspace, no allocation)."""
+    _check(library().lr_decode_attn_noalloc(
+        ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
+        _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, float(scale),
+        _ptr(o), _stream(stream)))
 
 
 def lr_topk_workspace_bytes(n_segments: int, T: int, k: int) -> int:
