@@ -40,37 +40,37 @@ using namespace sm100;
 constexpr int kHd = 128;
 constexpr int kChunk = 64;  // rank columns per ring stage
 constexpr int kStages = 3;
-constexpr int kThreads = 224;  // warp 0 TMA, 1 MMA, 2-5 epilogue, 6 residual rows
-constexpr int kEpi = 128;
+constexpr int kThreads = 352;  // warp 0 TMA, 1 MMA, 2-9 epilogue (two groups of 4), 10 residual rows
+constexpr int kEpi = 256;      // epilogue threads
+constexpr int kGrp = 128;      // threads of one epilogue group (one TMEM lane quarter per warp)
 
-constexpr uint32_t kColS1 = 0;
-constexpr uint32_t kColU = 256;
-constexpr uint32_t kColO3 = 384;
-constexpr uint32_t kColSC = 480;
+constexpr uint32_t kColS1 = 0;    // keys of both heads, fp32, 256 columns
+constexpr uint32_t kColU = 256;   // GELU-branch input of one 128-unit half
+constexpr uint32_t kColO3 = 384;  // per head slot: [sum p k~ | sum p g half0 | half1], 16 columns each
+constexpr uint32_t kColSC = 480;  // scores, hi and lo parts
 constexpr uint32_t kTmemCols = 512;
 
 template <int MG>
 struct Layout {
-  static constexpr uint32_t kQRows = 4 * MG;                      // Qhat rows: 2 heads x (hi, lo) x MG
-  static constexpr uint32_t kQBytes = kQRows * 128;               // one 64-column chunk of Qhat
-  static constexpr uint32_t kStageBytes = 49152 + kQBytes;        // A 16 KB, B_l 32 KB, Qhat
-  static constexpr uint32_t kStageTx = kStageBytes;
+  static constexpr uint32_t kQRows = 4 * MG;                  // Qhat rows: 2 heads x (hi, lo) x MG
+  static constexpr uint32_t kQBytes = kQRows * 128;           // one 64-column chunk of Qhat
+  static constexpr uint32_t kStageBytes = 49152 + kQBytes;    // A 16 KB, B_l 32 KB, Qhat
   static constexpr uint32_t kOffRing = 0;
-  static constexpr uint32_t kOffKt = (kStages * kStageBytes + 1023) & ~1023u;
+  static constexpr uint32_t kOffKt = (kStages * kStageBytes + 1023) & ~1023u;  // key tile of one head
   static constexpr uint32_t kOffG = kOffKt + 32768;
   static constexpr uint32_t kOffP = kOffG + 32768;
-  static constexpr uint32_t kOffB1 = kOffP + 4096;    // fp16 b1 of both heads (1 KB)
-  static constexpr uint32_t kOffRed = kOffB1 + 1024;  // 4 warps x 16 floats
-  static constexpr uint32_t kOffBar = kOffRed + 256;
+  static constexpr uint32_t kOffB1 = kOffP + 4096;      // fp16 b1 of both heads (1 KB)
+  static constexpr uint32_t kOffRed = kOffB1 + 1024;    // 4 warps x 16 floats
+  static constexpr uint32_t kOffAlpha = kOffRed + 256;  // [tile parity][head slot][8] softmax rescale
+  static constexpr uint32_t kOffBar = kOffAlpha + 128;
   static constexpr uint32_t kOffMisc = kOffBar + 256;
-  static constexpr uint32_t kOffAlpha = kOffMisc + 16;  // softmax rescale per (head slot, query head)
-  static constexpr uint32_t kSmemBytes = kOffMisc + 128 + 1024;  // + alignment slack
+  static constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 };
 static_assert(Layout<8>::kSmemBytes <= 232448, "shared memory budget");
 
 enum Bar {
-  FULL0 = 0, EMPTY0 = kStages, S1_FULL = 2 * kStages, S1_FREE, KT_READY, KT_FREE, U_FULL, U_FREE,
-  G_READY, G_FREE, O3_FULL0, O3_FULL1, O3_FREE0, O3_FREE1, DRAIN, EPI_SYNC, RES_READY, RES_DONE, N_BARS
+  FULL0 = 0, EMPTY0 = kStages, S1_FULL = 2 * kStages, S1_FREE, KT_READY, KT_FREE, U_FULL, U_FREE, G_READY,
+  G_FREE, O3_FULL0, O3_FULL1, O3_FREE0, O3_FREE1, EPI_SYNC, RES_READY, RES_DONE, DRAIN, N_BARS
 };
 static_assert(N_BARS * 8 <= 256, "barrier area");
 
@@ -159,77 +159,172 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col, uint32_t atom_by
   return a * atom_bytes + row * 128 + ((((c >> 3) ^ (row & 7))) << 4) + ((c & 7) << 1);
 }
 
-template <int MG>
-struct HeadState {
-  float m[MG], l[MG], ak[MG], ag0[MG], ag1[MG];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int g = 0; g < MG; ++g) {
-      m[g] = -CUDART_INF_F;
-      l[g] = ak[g] = ag0[g] = ag1[g] = 0.f;
-    }
-  }
-};
-
-struct EpiCtx {
-  int lq, ew, lane, row, tl, rmask;
-  uint32_t sync_phase;  // completed phases of the EPI_SYNC barrier
-  bool row_valid;
-  uint32_t trow;
-  uint8_t* sm;
-  uint64_t* bars;
-  volatile int* abort_flag;
-  size_t pseg;  // (b, layer, first head of the pair) segment index
-  TileInfo t;
-};
-
 // Epilogue-side wait: every lane polls, and the outcome is made uniform across the
 // warp so that a timeout never leaves part of a warp inside a collective.
 __device__ __forceinline__ bool ewait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
-// Barrier over the four epilogue warps, bounded like every other wait.
-__device__ __forceinline__ bool epi_sync(EpiCtx& c) {
-  mbar_arrive(&c.bars[EPI_SYNC]);
-  const bool ok = ewait(&c.bars[EPI_SYNC], c.sync_phase & 1, c.abort_flag);
-  ++c.sync_phase;
-  return ok;
-}
+template <int MG>
+struct Epi {
+  const TcArgs& a;
+  uint8_t* sm;
+  uint64_t* bars;
+  volatile int* abort_flag;
+  int grp, wl, lane, row;
+  uint32_t trow;
+  uint32_t sync_phase;
+  // group 0: softmax state and sum p k~; group 1: sum p g
+  float m[2][MG], l[2][MG], ak[2][MG], ag0[2][MG], ag1[2][MG];
+  float alpha[2][MG];
 
-// The epilogue's work for one KV head (slot HX of the pair) on the current tile.
-template <int HX, int MG>
-__device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<MG>& st) {
-  using L = Layout<MG>;
-  const int G = a.G, nh = a.H / 128;
-  uint64_t* bars = c.bars;
-  const uint4* b1h = reinterpret_cast<const uint4*>(c.sm + L::kOffB1 + HX * 512);
-  float* red = reinterpret_cast<float*>(c.sm + L::kOffRed);
-  uint8_t* ktile = c.sm + L::kOffKt;
-  uint8_t* gtile = c.sm + L::kOffG;
-  uint8_t* ptile = c.sm + L::kOffP;
-  const int row = c.row, lane = c.lane;
-  const int n_kt = 2 * c.tl + HX;
-  if (n_kt > 0 && !ewait(&bars[KT_FREE], (n_kt - 1) & 1, c.abort_flag)) return false;
-  // ---- scores (hi + lo columns) and the fp16 key tile
-  float sc[MG];
-  {
-    uint32_t sv[2 * MG];
-    if constexpr (MG == 4) {
-      uint32_t t8[8];
-      tmem_ld8(c.trow + kColSC + HX * 8, t8);
+  __device__ Epi(const TcArgs& a_, uint8_t* sm_, uint64_t* bars_, volatile int* ab, int warp, int lane_, uint32_t tmem)
+      : a(a_), sm(sm_), bars(bars_), abort_flag(ab) {
+    grp = (warp - 2) >> 2;
+    wl = (warp - 2) & 3;
+    lane = lane_;
+    const int lq = warp & 3;
+    row = lq * 32 + lane;
+    trow = tmem + ((uint32_t)(lq * 32) << 16);
+    sync_phase = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sv[i] = t8[i];
-    } else {
-      uint32_t t32[32];
-      tmem_ld32(c.trow + kColSC, t32);
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) sv[i] = t32[HX * 16 + i];
+      for (int g = 0; g < MG; ++g) {
+        m[h][g] = -CUDART_INF_F;
+        l[h][g] = ak[h][g] = ag0[h][g] = ag1[h][g] = 0.f;
+        alpha[h][g] = 1.f;
+      }
+  }
+
+  __device__ __forceinline__ bool sync0() {  // barrier over epilogue group 0
+    mbar_arrive(&bars[EPI_SYNC]);
+    const bool ok = ewait(&bars[EPI_SYNC], sync_phase & 1, abort_flag);
+    ++sync_phase;
+    return ok;
+  }
+
+  // Softmax of head slot HX on tile `tl` (group 0): scores -> p tile, alphas, KT_READY.
+  template <int HX>
+  __device__ __forceinline__ bool softmax(int tl, const float (&sc_in)[MG], bool hv) {
+    using L = Layout<MG>;
+    float* red = reinterpret_cast<float*>(sm + L::kOffRed);
+    uint8_t* ptile = sm + L::kOffP;
+    float sc[MG];
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      sc[g] = hv ? sc_in[g] : -CUDART_INF_F;
+      const float mx = warp_max(sc[g]);
+      if (lane == 0) red[wl * 16 + g] = mx;
     }
+    if (!sync0()) return false;
+    float p[MG];
+#pragma unroll
+    for (int g = 0; g < MG; ++g) {
+      const float mt = fmaxf(fmaxf(red[g], red[16 + g]), fmaxf(red[32 + g], red[48 + g]));
+      const float m_new = fmaxf(m[HX][g], mt);
+      alpha[HX][g] = m_new == -CUDART_INF_F ? 1.f : __expf(m[HX][g] - m_new);
+      p[g] = hv ? __expf(sc[g] - m_new) : 0.f;
+      l[HX][g] = l[HX][g] * alpha[HX][g] + p[g];
+      m[HX][g] = m_new;
+    }
+    // the p tile is free: the previous head's MMA3 (KT_FREE, waited before the key drain)
+    // and the residual warp are done with it
+    const int n_res = 2 * tl + HX;
+    if (n_res > 0 && !ewait(&bars[RES_DONE], (n_res - 1) & 1, abort_flag)) return false;
+#pragma unroll
+    for (int g = 0; g < MG; ++g)
+      if (g < a.G) *reinterpret_cast<__half*>(ptile + sw128_off(g, row, 2048)) = __float2half_rn(p[g]);
+    if (row == 0) {
+      float* al = reinterpret_cast<float*>(sm + L::kOffAlpha) + ((tl & 1) * 2 + HX) * 8;
+#pragma unroll
+      for (int g = 0; g < MG; ++g) al[g] = alpha[HX][g];
+    }
+    fence_proxy_async_smem();
+    if (!sync0()) return false;  // p tile and alphas complete; red consumed
+    mbar_arrive(&bars[KT_READY]);
+    if (row == 0) mbar_arrive(&bars[RES_READY]);
+    return true;
+  }
+
+  // GELU branch of head slot HX on tile `tl`: this group's 64 of every 128 hidden units.
+  template <int HX>
+  __device__ __forceinline__ bool gelu(int tl) {
+    using L = Layout<MG>;
+    const int nh = a.H / 128;
+    const uint4* b1h = reinterpret_cast<const uint4*>(sm + L::kOffB1 + HX * 512);
+    uint8_t* gtile = sm + L::kOffG;
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int half = 0; half < nh; ++half) {
+      const int j = (tl * 2 + HX) * nh + half;
+      if (!ewait(&bars[U_FULL], j & 1, abort_flag)) return false;
+      tc_fence_after();
+      uint32_t u[2][32];
+      tmem_ld32(trow + kColU + grp * 64, u[0]);
+      tmem_ld32(trow + kColU + grp * 64 + 32, u[1]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&bars[U_FREE]);
+      if (j > 0 && !ewait(&bars[G_FREE], (j - 1) & 1, abort_flag)) return false;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t* uu = &u[q >> 2][(q & 3) * 8];
+        const uint4 bb = b1h[half * 16 + grp * 8 + q];
+        uint4 w;
+        w.x = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[0]), __uint_as_float(uu[1])), bb.x));
+        w.y = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[2]), __uint_as_float(uu[3])), bb.y));
+        w.z = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[4]), __uint_as_float(uu[5])), bb.z));
+        w.w = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[6]), __uint_as_float(uu[7])), bb.w));
+        *reinterpret_cast<uint4*>(gtile + sw128_off(row, grp * 64 + q * 8, 16384)) = w;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars[G_READY]);
+    }
+    return true;
+  }
+
+  // Merge the tile's p-weighted sums of head slot HX into the running accumulators.
+  template <int HX>
+  __device__ __forceinline__ bool merge(int tl) {
+    using L = Layout<MG>;
+    if (!ewait(&bars[O3_FULL0 + HX], tl & 1, abort_flag)) return false;
+    tc_fence_after();
+    uint32_t v0[8], v1[8];
+    if (grp == 0) {
+      tmem_ld8(trow + kColO3 + HX * 48, v0);
+    } else {
+      tmem_ld8(trow + kColO3 + HX * 48 + 16, v0);
+      tmem_ld8(trow + kColO3 + HX * 48 + 32, v1);
+    }
+    tmem_ld_wait();
+    tc_fence_before();
+    mbar_arrive(&bars[O3_FREE0 + HX]);
+    if (grp == 0) {
+#pragma unroll
+      for (int g = 0; g < MG; ++g) ak[HX][g] = fmaf(ak[HX][g], alpha[HX][g], __uint_as_float(v0[g]));
+    } else {
+      // acquire group 0's alphas of this head (that phase has completed; the wait is immediate)
+      if (!ewait(&bars[KT_READY], (2 * tl + HX) & 1, abort_flag)) return false;
+      const float* al = reinterpret_cast<const float*>(sm + L::kOffAlpha) + ((tl & 1) * 2 + HX) * 8;
+#pragma unroll
+      for (int g = 0; g < MG; ++g) {
+        const float alg = al[g];
+        ag0[HX][g] = fmaf(ag0[HX][g], alg, __uint_as_float(v0[g]));
+        ag1[HX][g] = fmaf(ag1[HX][g], alg, __uint_as_float(v1[g]));
+      }
+    }
+    return true;
+  }
+
+  // Drain this group's 64 key columns of head slot HX into the fp16 key tile.
+  template <int HX>
+  __device__ __forceinline__ void drain() {
+    using L = Layout<MG>;
+    uint8_t* kt = sm + L::kOffKt;
+#pragma unroll 1
+    for (int cc = 0; cc < 2; ++cc) {
       uint32_t v[32];
-      tmem_ld32(c.trow + kColS1 + HX * 128 + cc * 32, v);
+      tmem_ld32(trow + kColS1 + HX * 128 + grp * 64 + cc * 32, v);
       tmem_ld_wait();
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -238,131 +333,104 @@ __device__ __forceinline__ bool epi_head(const TcArgs& a, EpiCtx& c, HeadState<M
         w.y = pack_f16x2_sat(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3]));
         w.z = pack_f16x2_sat(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5]));
         w.w = pack_f16x2_sat(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7]));
-        *reinterpret_cast<uint4*>(ktile + sw128_off(row, cc * 32 + q * 8, 16384)) = w;
+        *reinterpret_cast<uint4*>(kt + sw128_off(row, grp * 64 + cc * 32 + q * 8, 16384)) = w;
       }
     }
-#pragma unroll
-    for (int g = 0; g < MG; ++g) sc[g] = __uint_as_float(sv[g]) + __uint_as_float(sv[MG + g]);
   }
-  if (HX == 1) {
+
+  // One tile: for each head slot, drain its keys, then softmax, GELU branch and merge.
+  // The key tile is single-buffered: slot 1's keys stay in TMEM until slot 0 is done.
+  __device__ __forceinline__ bool tile(int tl, const TileInfo& t) {
+    const int half_row = row >> 6;
+    const int rblk = half_row ? t.blk[1] : t.blk[0];
+    const int tok = rblk * kBlock + (row & 63);
+    const bool row_valid = rblk >= 0 && tok < a.T;
+    const int rmask = half_row ? t.mask[1] : t.mask[0];
+    if (!ewait(&bars[S1_FULL], tl & 1, abort_flag)) return false;
+    tc_fence_after();
+    float sc[2][MG];
+    if (grp == 0) {  // scores of both heads (hi + lo columns)
+      uint32_t sv[32];
+      if constexpr (MG == 4) {
+        uint32_t t8[8];
+        tmem_ld8(trow + kColSC, t8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sv[i] = t8[i];
+        tmem_ld8(trow + kColSC + 8, t8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sv[16 + i] = t8[i];
+      } else {
+        tmem_ld32(trow + kColSC, sv);
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int g = 0; g < MG; ++g) {
+        sc[0][g] = __uint_as_float(sv[g]) + __uint_as_float(sv[MG + g]);
+        sc[1][g] = MG == 4 ? __uint_as_float(sv[16 + g]) + __uint_as_float(sv[16 + MG + g])
+                           : __uint_as_float(sv[2 * MG + g]) + __uint_as_float(sv[3 * MG + g]);
+      }
+    }
+    const bool hv0 = row_valid && (rmask & 1), hv1 = row_valid && ((rmask >> 1) & 1);
+    // ---- head slot 0
+    if (tl > 0 && !ewait(&bars[KT_FREE], (2 * tl - 1) & 1, abort_flag)) return false;
+    drain<0>();
+    fence_proxy_async_smem();
+    if (grp == 1) mbar_arrive(&bars[KT_READY]);
+    if (grp == 0 && !softmax<0>(tl, sc[0], hv0)) return false;
+    if (!gelu<0>(tl)) return false;
+    if (!merge<0>(tl)) return false;
+    // ---- head slot 1 (its keys leave TMEM now, which frees S1 for the next tile)
+    if (!ewait(&bars[KT_FREE], (2 * tl) & 1, abort_flag)) return false;
+    drain<1>();
     tc_fence_before();
     mbar_arrive(&bars[S1_FREE]);
-  }
-  // ---- online softmax over the tile
-  const bool hv = c.row_valid && ((c.rmask >> HX) & 1);
-  float alpha[MG], p[MG];
-#pragma unroll
-  for (int g = 0; g < MG; ++g) {
-    if (!hv) sc[g] = -CUDART_INF_F;
-    const float m = warp_max(sc[g]);
-    if (lane == 0) red[c.ew * 16 + g] = m;
-  }
-  if (!epi_sync(c)) return false;
-#pragma unroll
-  for (int g = 0; g < MG; ++g) {
-    const float mt = fmaxf(fmaxf(red[g], red[16 + g]), fmaxf(red[32 + g], red[48 + g]));
-    const float m_new = fmaxf(st.m[g], mt);
-    alpha[g] = m_new == -CUDART_INF_F ? 1.f : __expf(st.m[g] - m_new);
-    p[g] = hv ? __expf(sc[g] - m_new) : 0.f;
-    st.l[g] = st.l[g] * alpha[g] + p[g];
-    st.m[g] = m_new;
-  }
-  // the residual warp has finished with the previous head's p tile
-  if (n_kt > 0 && !ewait(&bars[RES_DONE], (n_kt - 1) & 1, c.abort_flag)) return false;
-#pragma unroll
-  for (int g = 0; g < MG; ++g)
-    if (g < G) *reinterpret_cast<__half*>(ptile + sw128_off(g, row, 2048)) = __float2half_rn(p[g]);
-  if (row == 0) {
-    float* al = reinterpret_cast<float*>(c.sm + L::kOffAlpha) + HX * 8;
-#pragma unroll
-    for (int g = 0; g < MG; ++g) al[g] = alpha[g];
-  }
-  fence_proxy_async_smem();
-  if (!epi_sync(c)) return false;  // p tile and alpha complete; red consumed
-  mbar_arrive(&bars[KT_READY]);
-  if (row == 0) mbar_arrive(&bars[RES_READY]);
-  // ---- GELU branch, one 128-unit half at a time
-#pragma unroll 1
-  for (int half = 0; half < nh; ++half) {
-    const int j = n_kt * nh + half;
-    if (!ewait(&bars[U_FULL], j & 1, c.abort_flag)) return false;
-    tc_fence_after();
-    uint32_t u[4][32];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld32(c.trow + kColU + q * 32, u[q]);
-    tmem_ld_wait();
-    tc_fence_before();
-    mbar_arrive(&bars[U_FREE]);
-    if (j > 0 && !ewait(&bars[G_FREE], (j - 1) & 1, c.abort_flag)) return false;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const uint32_t* uu = &u[q >> 2][(q & 3) * 8];
-      const uint4 bb = b1h[half * 16 + q];
-      uint4 w;
-      w.x = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[0]), __uint_as_float(uu[1])), bb.x));
-      w.y = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[2]), __uint_as_float(uu[3])), bb.y));
-      w.z = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[4]), __uint_as_float(uu[5])), bb.z));
-      w.w = gelu_f16x2(add_f16x2(pack_f16x2_sat(__uint_as_float(uu[6]), __uint_as_float(uu[7])), bb.w));
-      *reinterpret_cast<uint4*>(gtile + sw128_off(row, q * 8, 16384)) = w;
-    }
     fence_proxy_async_smem();
-    mbar_arrive(&bars[G_READY]);
+    if (grp == 1) mbar_arrive(&bars[KT_READY]);
+    if (grp == 0 && !softmax<1>(tl, sc[1], hv1)) return false;
+    if (!gelu<1>(tl)) return false;
+    if (!merge<1>(tl)) return false;
+    return true;
   }
-  // ---- merge this tile's p-weighted sums (O3 lane = dim `row`)
-  if (!ewait(&bars[O3_FULL0 + HX], c.tl & 1, c.abort_flag)) return false;
-  tc_fence_after();
-  uint32_t ok8[8], og0[8], og1[8];
-  tmem_ld8(c.trow + kColO3 + HX * 48, ok8);
-  tmem_ld8(c.trow + kColO3 + HX * 48 + 16, og0);
-  tmem_ld8(c.trow + kColO3 + HX * 48 + 32, og1);
-  tmem_ld_wait();
-  tc_fence_before();
-  mbar_arrive(&bars[O3_FREE0 + HX]);
-#pragma unroll
-  for (int g = 0; g < MG; ++g) {
-    st.ak[g] = fmaf(st.ak[g], alpha[g], __uint_as_float(ok8[g]));
-    st.ag0[g] = fmaf(st.ag0[g], alpha[g], __uint_as_float(og0[g]));
-    st.ag1[g] = fmaf(st.ag1[g], alpha[g], __uint_as_float(og1[g]));
-  }
-  return true;
-}
 
-template <int MG>
-__device__ __forceinline__ void write_partials(const TcArgs& a, EpiCtx& c, const HeadState<MG>& s0,
-                                               const HeadState<MG>& s1, int b, int split, int ha) {
-  using L = Layout<MG>;
-  float* red = reinterpret_cast<float*>(c.sm + L::kOffRed);
-  epi_sync(c);  // red is free
+  __device__ __forceinline__ void write_partials(int b, int split, int ha) {
+    using L = Layout<MG>;
+    float* red = reinterpret_cast<float*>(sm + L::kOffRed);
+    const int Hq = a.Hkv * a.G;
+    if (grp == 0) {
+      sync0();  // red is free
 #pragma unroll
-  for (int g = 0; g < MG; ++g) {
-    const float v0 = warp_sum(s0.l[g]);
-    const float v1 = warp_sum(s1.l[g]);
-    if (c.lane == 0) {
-      red[c.ew * 16 + g] = v0;
-      red[c.ew * 16 + 8 + g] = v1;
-    }
-  }
-  epi_sync(c);
-  const int Hq = a.Hkv * a.G, row = c.row;
-#pragma unroll
-  for (int hx = 0; hx < 2; ++hx) {
-    const HeadState<MG>& st = hx ? s1 : s0;
-#pragma unroll
-    for (int g = 0; g < MG; ++g) {
-      if (g >= a.G) continue;
-      const int hq = (ha + hx) * a.G + g;
-      float* part = a.partials + (((size_t)b * Hq + hq) * a.n_split + split) * a.part_stride;
-      if (row == 0) {
-        part[0] = st.m[g];
-        part[1] = red[hx * 8 + g] + red[16 + hx * 8 + g] + red[32 + hx * 8 + g] + red[48 + hx * 8 + g];
-        part[2] = part[3] = 0.f;
+      for (int g = 0; g < MG; ++g) {
+        const float v0 = warp_sum(l[0][g]);
+        const float v1 = warp_sum(l[1][g]);
+        if (lane == 0) {
+          red[wl * 16 + g] = v0;
+          red[wl * 16 + 8 + g] = v1;
+        }
       }
-      part[4 + row] = st.ak[g];
-      part[4 + kHd + row] = st.ag0[g];
-      if (a.H == 256) part[4 + kHd + 128 + row] = st.ag1[g];
+      sync0();
+    }
+#pragma unroll
+    for (int hx = 0; hx < 2; ++hx) {
+#pragma unroll
+      for (int g = 0; g < MG; ++g) {
+        if (g >= a.G) continue;
+        const int hq = (ha + hx) * a.G + g;
+        float* part = a.partials + (((size_t)b * Hq + hq) * a.n_split + split) * a.part_stride;
+        if (grp == 0) {
+          if (row == 0) {
+            part[0] = m[hx][g];
+            part[1] = red[hx * 8 + g] + red[16 + hx * 8 + g] + red[32 + hx * 8 + g] + red[48 + hx * 8 + g];
+            part[2] = part[3] = 0.f;
+          }
+          part[4 + row] = ak[hx][g];
+        } else {
+          part[4 + kHd + row] = ag0[hx][g];
+          if (a.H == 256) part[4 + kHd + 128 + row] = ag1[hx][g];
+        }
+      }
     }
   }
-}
+};
 
 // The residual warp: for each (tile, head) it scatters p_t r_t over the residual rows of the
 // tile's blocks ("Predicting the value cache from keys", paragraph 2). Lane l owns dims
@@ -444,7 +512,7 @@ __device__ __forceinline__ void residual_warp(const TcArgs& a, uint8_t* sm, uint
           waited = true;
 #pragma unroll
           for (int g = 0; g < MG; ++g) {
-            const float al = alphas[hx * 8 + g];
+            const float al = alphas[((tl & 1) * 2 + hx) * 8 + g];
 #pragma unroll
             for (int d = 0; d < 4; ++d) acc[hx][g][d] *= al;
           }
@@ -511,7 +579,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
 
   const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int H = a.H, nh = a.H / 128, nk = a.r / kChunk;
+  const int H = a.H, nh = a.H / 128, nk = a.r / kChunk, nw = 2 * nh;
   const int n_tiles = tile_count(a, b, hp);
   const int t_begin = (int)((long long)s * n_tiles / a.n_split);
   const int t_end = (int)((long long)(s + 1) * n_tiles / a.n_split);
@@ -535,10 +603,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
     mbar_init(&bars[O3_FULL1], 1);
     mbar_init(&bars[O3_FREE0], kEpi);
     mbar_init(&bars[O3_FREE1], kEpi);
-    mbar_init(&bars[DRAIN], 1);
-    mbar_init(&bars[EPI_SYNC], kEpi);
+    mbar_init(&bars[EPI_SYNC], kGrp);
     mbar_init(&bars[RES_READY], 1);
     mbar_init(&bars[RES_DONE], 1);
+    mbar_init(&bars[DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -585,23 +653,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
           const uint32_t st = it % kStages, ph = (it / kStages) & 1;
           if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
           uint8_t* dst = sm + L::kOffRing + st * L::kStageBytes;
-          mbar_arrive_expect_tx(&bars[FULL0 + st], L::kStageTx);
+          mbar_arrive_expect_tx(&bars[FULL0 + st], L::kStageBytes);
           tma_load_3d(dst, &mapA, &bars[FULL0 + st], kc * kChunk, row0, b);
           tma_load_3d(dst + 8192, &mapA, &bars[FULL0 + st], kc * kChunk, row1, b);
           tma_load_3d(dst + 16384, &mapB, &bars[FULL0 + st], kc * kChunk, rowB, b);
           tma_load_3d(dst + 32768, &mapB, &bars[FULL0 + st], kc * kChunk, rowB + kHd, b);
           tma_load_2d(dst + 49152, &mapQ, &bars[FULL0 + st], kc * kChunk, rowQ);
         }
-        for (int hx = 0; hx < 2 && ok; ++hx) {
-          for (int half = 0; half < nh && ok; ++half, ++it) {
-            const uint32_t st = it % kStages, ph = (it / kStages) & 1;
-            if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
-            uint8_t* dst = sm + L::kOffRing + st * L::kStageBytes;
-            const int wrow = ((w1seq * a.Hkv + ha + hx) * H) + half * 128;
-            mbar_arrive_expect_tx(&bars[FULL0 + st], 32768);
-            tma_load_2d(dst, &mapW1, &bars[FULL0 + st], 0, wrow);
-            tma_load_2d(dst + 16384, &mapW1, &bars[FULL0 + st], 64, wrow);
-          }
+        for (int j = 0; j < nw && ok; ++j, ++it) {
+          const int hx = j / nh, half = j % nh;
+          const uint32_t st = it % kStages, ph = (it / kStages) & 1;
+          if (!(ok = mbar_wait(&bars[EMPTY0 + st], ph ^ 1, abort_flag))) break;
+          uint8_t* dst = sm + L::kOffRing + st * L::kStageBytes;
+          const int wrow = ((w1seq * a.Hkv + ha + hx) * H) + half * 128;
+          mbar_arrive_expect_tx(&bars[FULL0 + st], 32768);
+          tma_load_2d(dst, &mapW1, &bars[FULL0 + st], 0, wrow);
+          tma_load_2d(dst + 16384, &mapW1, &bars[FULL0 + st], 64, wrow);
         }
       }
       if (!ok) {
@@ -689,45 +756,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
       mma_commit(&bars[DRAIN]);
       mbar_wait_drain(&bars[DRAIN], 0, kWaitCycles / 4);
     }
-  } else if (warp == 6) {
+  } else if (warp == 10) {
     // ---------------------------------------------------------------- residual rows
     residual_warp<MG>(a, sm, bars, abort_flag, b, hp, s, t_begin, t_end);
   } else {
-    // ---------------------------------------------------------------- epilogue
-    EpiCtx c;
-    c.lq = warp & 3;
-    c.ew = warp - 2;
-    c.lane = lane;
-    c.row = c.lq * 32 + lane;
-    c.trow = tmem + ((uint32_t)(c.lq * 32) << 16);
-    c.sm = sm;
-    c.bars = bars;
-    c.abort_flag = abort_flag;
-    c.sync_phase = 0;
-    c.pseg = ((size_t)b * a.L + a.layer) * a.Hkv + ha;
-    HeadState<MG> st0, st1;
-    st0.init();
-    st1.init();
+    // ---------------------------------------------------------------- epilogue (warps 2-9)
+    Epi<MG> e(a, sm, bars, abort_flag, warp, lane, tmem);
     bool ok = true;
-    int tl = 0;
-    for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
-      c.t = tile_info(a, b, hp, ti);
-      const int half_row = c.row >> 6;
-      const int rblk = half_row ? c.t.blk[1] : c.t.blk[0];
-      const int tok = rblk * kBlock + (c.row & 63);
-      c.row_valid = rblk >= 0 && tok < a.T;
-      c.rmask = half_row ? c.t.mask[1] : c.t.mask[0];
-      c.tl = tl;
-      if (!(ok = ewait(&bars[S1_FULL], tl & 1, abort_flag))) break;
-      tc_fence_after();
-      ok = epi_head<0, MG>(a, c, st0);
-      if (ok) ok = epi_head<1, MG>(a, c, st1);
-    }
+    for (int i = 0; t_begin + i < t_end && ok; ++i) ok = e.tile(i, tile_info(a, b, hp, t_begin + i));
     if (!ok) {
       *abort_flag = 1;
       flag_error(a.err, LR_DEVERR_TIMEOUT);
     }
-    write_partials<MG>(a, c, st0, st1, b, s, ha);
+    e.write_partials(b, s, ha);
   }
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
