@@ -196,39 +196,58 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
     }
   }
   __syncthreads();
+  // weighted sums over the splits, 8 independent loads in flight per step
   for (int x = tid; x < G * W; x += CT) {
     const int g = x / W, e = x % W;
     const float* part = part0 + (size_t)g * S * a.part_stride + 4 + e;
     const float* wg = wsplit + g * S;
-    float v = 0.f;
-    for (int s = 0; s < S; ++s) v = fmaf(wg[s], part[(size_t)s * a.part_stride], v);
-    accs[x] = v;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int s = 0;
+    for (; s + 8 <= S; s += 8) {
+      float t[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) t[u] = part[(size_t)(s + u) * a.part_stride];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = fmaf(wg[s + u], t[u], v[u]);
+    }
+    for (; s < S; ++s) v[0] = fmaf(wg[s], part[(size_t)s * a.part_stride], v[0]);
+    accs[x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
   }
   __syncthreads();
   const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, h);
   T* o = (T*)a.o + ((size_t)b * Hq + (size_t)h * G) * hd;
-  for (int j = warp; j < hd; j += CT / 32) {
-    const T* wl = P.W_lin + (size_t)j * hd;
-    const T* w2 = P.W2 + (size_t)j * H;
-    float wlv[8], w2v[16];
+  for (int j0 = warp; j0 < hd; j0 += 2 * (CT / 32)) {
+    float wlv[2][8], w2v[2][16], bj[2];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) wlv[q] = lane + 32 * q < hd ? to_f32(wl[lane + 32 * q]) : 0.f;
+    for (int r = 0; r < 2; ++r) {
+      const int j = j0 + r * (CT / 32);
+      const bool on = j < hd;
+      const T* wl = P.W_lin + (size_t)(on ? j : 0) * hd;
+      const T* w2 = P.W2 + (size_t)(on ? j : 0) * H;
 #pragma unroll
-    for (int q = 0; q < 16; ++q) w2v[q] = lane + 32 * q < H ? to_f32(w2[lane + 32 * q]) : 0.f;
-    const float bj = P.b2 ? to_f32(P.b2[j]) : 0.f;
-    for (int g = 0; g < G; ++g) {
-      const float* ac = accs + g * W;
-      float y = 0.f;
+      for (int q = 0; q < 8; ++q) wlv[r][q] = (on && lane + 32 * q < hd) ? to_f32(wl[lane + 32 * q]) : 0.f;
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q < hd) y = fmaf(ac[lane + 32 * q], wlv[q], y);
+      for (int q = 0; q < 16; ++q) w2v[r][q] = (on && lane + 32 * q < H) ? to_f32(w2[lane + 32 * q]) : 0.f;
+      bj[r] = (on && P.b2) ? to_f32(P.b2[j]) : 0.f;
+    }
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
-        if (lane + 32 * q < H) y = fmaf(ac[hd + lane + 32 * q], w2v[q], y);
-      y = warp_sum(y);
-      if (lane == 0) {
-        const float out = mx[g] == -CUDART_INF_F ? 0.f : (y + ac[hd + H + j]) * inv_l[g] + bj;
-        o[(size_t)g * hd + j] = from_f32<T>(out);
+    for (int r = 0; r < 2; ++r) {
+      const int j = j0 + r * (CT / 32);
+      if (j >= hd) continue;
+      for (int g = 0; g < G; ++g) {
+        const float* ac = accs + g * W;
+        float y = 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (lane + 32 * q < hd) y = fmaf(ac[lane + 32 * q], wlv[r][q], y);
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (lane + 32 * q < H) y = fmaf(ac[hd + lane + 32 * q], w2v[r][q], y);
+        y = warp_sum(y);
+        if (lane == 0) {
+          const float out = mx[g] == -CUDART_INF_F ? 0.f : (y + ac[hd + H + j]) * inv_l[g] + bj[r];
+          o[(size_t)g * hd + j] = from_f32<T>(out);
+        }
       }
     }
   }

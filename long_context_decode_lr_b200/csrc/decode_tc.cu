@@ -713,6 +713,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
           if (!(ok = mbar_wait(&bars[KT_READY], n_kt & 1, abort_flag))) break;
           if (!(ok = mbar_wait(&bars[O3_FREE0 + hx], (tl & 1) ^ 1, abort_flag))) break;
           tc_fence_after();
+          // sum p k~ needs only the key and p tiles: issue it ahead of the GELU branch
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16_ss(tmem + kColO3 + hx * 48, sw128_desc(kt + ks * 2048, 16384, 1024),
+                       sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
           for (int half = 0; half < nh && ok; ++half, ++it) {
             const int j = n_kt * nh + half;
             const uint32_t st = it % kStages, ph = (it / kStages) & 1;
@@ -740,10 +745,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
             mma_commit(&bars[G_FREE]);
           }
           if (!ok) break;
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_f16_ss(tmem + kColO3 + hx * 48, sw128_desc(kt + ks * 2048, 16384, 1024),
-                       sw128_desc(pt + (ks >> 2) * 2048 + (ks & 3) * 32, 16, 1024), id_o3, ks != 0);
           mma_commit(&bars[KT_FREE]);
           mma_commit(&bars[O3_FULL0 + hx]);
         }
@@ -785,7 +786,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
 //                                2^-14 or above 65504, where values saturate)
 //   blocks [n_w1, n_w1 + n_q)    Qhat = scale * B_l^h q for every query head, stored as bf16
 //                                hi + lo rows (hi = bf16(x), lo = bf16(x - hi)); one block per
-//                                (256 rank columns, KV head, sequence)
+//                                (64 rank columns, KV head, sequence)
 //   blocks [n_w1 + n_q, ...)     selective mode: per (sequence, head pair) the union of the two
 //                                block lists with a 2-bit head mask (bit 0: first head); entries
 //                                out of range or not strictly ascending are skipped and flagged
@@ -809,8 +810,11 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(TcArgs a, int n_w1,
     return;
   }
   if (bid < n_w1 + n_q) {
+    // one block per (64 rank columns, KV head, sequence): thread (dg, c) sums 32 of the 128
+    // key dims for column c, all loads of a thread in flight at once; then a 4-way reduction
     __shared__ float qs[8][kHd];
-    const int nj = (a.r + 255) / 256;
+    __shared__ float part[4][64][MG];
+    const int nj = (a.r + 63) / 64;
     const int q = bid - n_w1;
     const int jc = q % nj, h = (q / nj) % a.Hkv, b = q / (nj * a.Hkv);
     const int G = a.G;
@@ -819,25 +823,34 @@ __global__ void __launch_bounds__(256) decode_tc_prep_kernel(TcArgs a, int n_w1,
       qs[g][d] = g < G ? __bfloat162float(a.q[(((size_t)b * a.Hkv + h) * G + g) * kHd + d]) * a.scale : 0.f;
     }
     __syncthreads();
-    const int j = jc * 256 + tid;
-    if (j >= a.r) return;
-    const size_t D = (size_t)a.L * a.Hkv * kHd;
-    const __nv_bfloat16* bt = a.Bt + (size_t)b * D * a.r + ((size_t)(a.layer * a.Hkv + h) * kHd) * a.r + j;
+    const int c = tid & 63, dg = tid >> 6;
+    const int j = jc * 64 + c;
     float acc[MG];
 #pragma unroll
     for (int g = 0; g < MG; ++g) acc[g] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < kHd; ++d) {
-      const float v = __bfloat162float(bt[(size_t)d * a.r]);
+    if (j < a.r) {
+      const size_t D = (size_t)a.L * a.Hkv * kHd;
+      const __nv_bfloat16* bt =
+          a.Bt + (size_t)b * D * a.r + ((size_t)(a.layer * a.Hkv + h) * kHd + dg * 32) * a.r + j;
+      float v[32];
 #pragma unroll
-      for (int g = 0; g < MG; ++g) acc[g] = fmaf(v, qs[g][d], acc[g]);
+      for (int d = 0; d < 32; ++d) v[d] = __bfloat162float(bt[(size_t)d * a.r]);
+#pragma unroll
+      for (int d = 0; d < 32; ++d)
+#pragma unroll
+        for (int g = 0; g < MG; ++g) acc[g] = fmaf(v[d], qs[g][dg * 32 + d], acc[g]);
     }
+#pragma unroll
+    for (int g = 0; g < MG; ++g) part[dg][c][g] = acc[g];
+    __syncthreads();
+    if (dg != 0 || j >= a.r) return;
     const int hp = h >> 1, hx = h & 1;
     __nv_bfloat16* out = a.qhat + ((size_t)(b * a.n_hp + hp) * (4 * MG) + hx * 2 * MG) * a.r + j;
 #pragma unroll
     for (int g = 0; g < MG; ++g) {
-      const __nv_bfloat16 hi = __float2bfloat16_rn(acc[g]);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(acc[g] - __bfloat162float(hi));
+      const float x = part[0][c][g] + part[1][c][g] + part[2][c][g] + part[3][c][g];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
       out[(size_t)g * a.r] = hi;
       out[(size_t)(MG + g) * a.r] = lo;
     }
@@ -881,7 +894,7 @@ cudaError_t launch_mg(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap&
                       const CUtensorMap& mW1, const int* blocks, int n_sel, cudaStream_t st) {
   const size_t n_w1_vec = (size_t)a.w1_seqs * a.Hkv * a.H * kHd / 4;
   const int n_w1 = (int)((n_w1_vec + 255) / 256 < 512 ? (n_w1_vec + 255) / 256 : 512);
-  const int n_q = ((a.r + 255) / 256) * a.Hkv * a.B;
+  const int n_q = ((a.r + 63) / 64) * a.Hkv * a.B;
   const int n_s = a.sched ? a.n_hp * a.B : 0;
   decode_tc_prep_kernel<MG><<<n_w1 + n_q + n_s, 256, 0, st>>>(a, n_w1, n_q, blocks, n_sel);
   cudaError_t e = cudaGetLastError();
