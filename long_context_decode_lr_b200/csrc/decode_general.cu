@@ -160,95 +160,121 @@ __global__ void __launch_bounds__(NT) decode_general_kernel(DecodeArgs a) {
   }
 }
 
-// Merge the split partials of the G query heads of one (sequence, KV head) and apply
-// the linear maps once per query head: o = (acc_k W_lin^T + acc_g W2^T + acc_r) / l + b2.
-// Partial sums are read coalesced (threads over entries); each output element is a
-// warp-wide dot product over a contiguous weight row.
-constexpr int CT = 512;  // combine threads
+// Merge the split partials of one query head and apply the linear maps once:
+// o = (acc_k W_lin^T + acc_g W2^T + acc_r) / l + b2. One block per (chunk of CJ output
+// columns, query head, sequence), so that even a single sequence spreads over many SMs;
+// every block of a head re-merges acc_k and acc_g (hd + H floats per split, read from
+// L2) and only its own CJ columns of acc_r. The kernel may start while the split kernel
+// drains (programmatic dependent launch): it stages its weight rows in shared memory
+// first, then waits for the split kernel before the first partial is read. The merge
+// runs over (entry, split chunk) items so that each thread keeps eight loads in flight,
+// and the chunk sums are added in a fixed order.
+constexpr int CT = 512;      // combine threads
+constexpr int CJ = 32;       // output columns per combine block
+constexpr int kMaxChunk = 8; // split chunks per merged entry
+
+struct CombineSmem {
+  int n_ch, cs, n_acc, w_floats;
+  int off_ml, off_w, off_red, off_acc, total;  // in floats
+};
+
+__host__ __device__ inline CombineSmem combine_smem(int hd, int H, int S, int elem_bytes) {
+  CombineSmem c;
+  c.n_ch = ceil_div(S, 8) < kMaxChunk ? ceil_div(S, 8) : kMaxChunk;
+  c.cs = ceil_div(S, c.n_ch);
+  c.n_acc = hd + H + CJ;
+  c.w_floats = ceil_div(CJ * (hd + H) * elem_bytes, 16) * 4;  // weight rows, 16-byte padded
+  c.off_w = 0;
+  c.off_ml = c.w_floats;
+  c.off_red = c.off_ml + 2 * S;
+  c.off_acc = c.off_red + c.n_ch * c.n_acc;
+  c.total = c.off_acc + c.n_acc;
+  return c;
+}
 
 template <typename T>
 __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
   extern __shared__ float sm[];
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hd = a.hd, H = a.H, G = a.G, Hq = a.Hkv * a.G, S = a.n_split, W = 2 * hd + H;
-  float* wsplit = sm;              // [G][S]
-  float* accs = wsplit + G * S;    // [G][W]
-  float* inv_l = accs + G * W;     // [G]
-  float* mx = inv_l + G;           // [G]
-  const float* part0 = a.partials + ((size_t)b * Hq + (size_t)h * G) * S * a.part_stride;
-  // split maxima and weights, one warp per query head
-  for (int g = warp; g < G; g += CT / 32) {
-    const float* part = part0 + (size_t)g * S * a.part_stride;
+  __shared__ float s_m, s_inv_l, s_b2[CJ];
+  const int jc = blockIdx.x, qh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int hd = a.hd, H = a.H, Hq = a.Hkv * a.G, S = a.n_split;
+  const int j0 = jc * CJ, nj = min(CJ, hd - j0);
+  const CombineSmem L = combine_smem(hd, H, S, (int)sizeof(T));
+  T* wl_s = reinterpret_cast<T*>(sm + L.off_w);  // [nj][hd]
+  T* w2_s = wl_s + CJ * hd;                      // [nj][H]
+  float* mls = sm + L.off_ml;                    // [S] maxima, then [S] sums
+  float* red = sm + L.off_red;                   // [n_ch][n_acc]
+  float* acc = sm + L.off_acc;                   // [hd + H + nj]: merged sum p k~, sum p g, own columns of sum p r
+
+  // weight rows are inputs of the call, independent of the split kernel
+  const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, qh / a.G);
+  for (int i = tid; i < nj * hd; i += CT) wl_s[i] = P.W_lin[(size_t)j0 * hd + i];
+  for (int i = tid; i < nj * H; i += CT) w2_s[i] = P.W2[(size_t)j0 * H + i];
+  if (tid < nj) s_b2[tid] = P.b2 ? to_f32(P.b2[j0 + tid]) : 0.f;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const float* part = a.partials + ((size_t)b * Hq + qh) * S * a.part_stride;
+  for (int s = tid; s < S; s += CT) {
+    mls[s] = part[(size_t)s * a.part_stride];
+    mls[S + s] = part[(size_t)s * a.part_stride + 1];
+  }
+  __syncthreads();
+  if (warp == 0) {
     float m = -CUDART_INF_F;
-    for (int s = lane; s < S; s += 32) m = fmaxf(m, part[(size_t)s * a.part_stride]);
+    for (int s = lane; s < S; s += 32) m = fmaxf(m, mls[s]);
     m = warp_max(m);
     float l = 0.f;
     for (int s = lane; s < S; s += 32) {
-      const float ms = part[(size_t)s * a.part_stride];
+      const float ms = mls[s];
       const float wgt = (m == -CUDART_INF_F || ms == -CUDART_INF_F) ? 0.f : __expf(ms - m);
-      wsplit[g * S + s] = wgt;
-      l = fmaf(wgt, part[(size_t)s * a.part_stride + 1], l);
+      mls[s] = wgt;
+      l = fmaf(wgt, mls[S + s], l);
     }
     l = warp_sum(l);
     if (lane == 0) {
-      mx[g] = m;
-      inv_l[g] = l > 0.f ? 1.f / l : 0.f;
+      s_m = m;
+      s_inv_l = l > 0.f ? 1.f / l : 0.f;
     }
   }
   __syncthreads();
-  // weighted sums over the splits, 8 independent loads in flight per step
-  for (int x = tid; x < G * W; x += CT) {
-    const int g = x / W, e = x % W;
-    const float* part = part0 + (size_t)g * S * a.part_stride + 4 + e;
-    const float* wg = wsplit + g * S;
+  const int n_acc = hd + H + nj;
+  for (int it = tid; it < L.n_ch * n_acc; it += CT) {
+    const int c = it / n_acc, x = it % n_acc;
+    const int e = x < hd + H ? x : x + j0;
+    const int s0 = c * L.cs, s1 = min(S, s0 + L.cs);
+    const float* pe = part + 4 + e;
     float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int s = 0;
-    for (; s + 8 <= S; s += 8) {
+    int s = s0;
+    for (; s + 8 <= s1; s += 8) {
       float t[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) t[u] = part[(size_t)(s + u) * a.part_stride];
+      for (int u = 0; u < 8; ++u) t[u] = pe[(size_t)(s + u) * a.part_stride];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = fmaf(wg[s + u], t[u], v[u]);
+      for (int u = 0; u < 8; ++u) v[u] = fmaf(mls[s + u], t[u], v[u]);
     }
-    for (; s < S; ++s) v[0] = fmaf(wg[s], part[(size_t)s * a.part_stride], v[0]);
-    accs[x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
+    for (; s < s1; ++s) v[0] = fmaf(mls[s], pe[(size_t)s * a.part_stride], v[0]);
+    red[c * L.n_acc + x] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
   }
   __syncthreads();
-  const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, h);
-  T* o = (T*)a.o + ((size_t)b * Hq + (size_t)h * G) * hd;
-  for (int j0 = warp; j0 < hd; j0 += 2 * (CT / 32)) {
-    float wlv[2][8], w2v[2][16], bj[2];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int j = j0 + r * (CT / 32);
-      const bool on = j < hd;
-      const T* wl = P.W_lin + (size_t)(on ? j : 0) * hd;
-      const T* w2 = P.W2 + (size_t)(on ? j : 0) * H;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) wlv[r][q] = (on && lane + 32 * q < hd) ? to_f32(wl[lane + 32 * q]) : 0.f;
-#pragma unroll
-      for (int q = 0; q < 16; ++q) w2v[r][q] = (on && lane + 32 * q < H) ? to_f32(w2[lane + 32 * q]) : 0.f;
-      bj[r] = (on && P.b2) ? to_f32(P.b2[j]) : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int j = j0 + r * (CT / 32);
-      if (j >= hd) continue;
-      for (int g = 0; g < G; ++g) {
-        const float* ac = accs + g * W;
-        float y = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (lane + 32 * q < hd) y = fmaf(ac[lane + 32 * q], wlv[r][q], y);
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (lane + 32 * q < H) y = fmaf(ac[hd + lane + 32 * q], w2v[r][q], y);
-        y = warp_sum(y);
-        if (lane == 0) {
-          const float out = mx[g] == -CUDART_INF_F ? 0.f : (y + ac[hd + H + j]) * inv_l[g] + bj[r];
-          o[(size_t)g * hd + j] = from_f32<T>(out);
-        }
-      }
+  for (int x = tid; x < n_acc; x += CT) {
+    float v = 0.f;
+    for (int c = 0; c < L.n_ch; ++c) v += red[c * L.n_acc + x];
+    acc[x] = v;
+  }
+  __syncthreads();
+  T* o = (T*)a.o + ((size_t)b * Hq + qh) * hd;
+  const float m = s_m, inv_l = s_inv_l;
+  for (int jj = warp; jj < nj; jj += CT / 32) {
+    const T* wl = wl_s + jj * hd;
+    const T* w2 = w2_s + jj * H;
+    float y0 = 0.f, y1 = 0.f;
+    for (int c = lane; c < hd; c += 32) y0 = fmaf(acc[c], to_f32(wl[c]), y0);
+    for (int c = lane; c < H; c += 32) y1 = fmaf(acc[hd + c], to_f32(w2[c]), y1);
+    const float y = warp_sum(y0 + y1);
+    if (lane == 0) {
+      const float out = m == -CUDART_INF_F ? 0.f : (y + acc[hd + H + jj]) * inv_l + s_b2[jj];
+      o[j0 + jj] = from_f32<T>(out);
     }
   }
 }
@@ -259,8 +285,9 @@ size_t decode_general_smem_bytes(int hd, int H, int G) {
   return (size_t)decode_smem_plan(hd, H, G).total * sizeof(float);
 }
 
-size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split) {
-  return (size_t)(G * n_split + G * (2 * hd + H) + 2 * G) * sizeof(float);
+size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split, int elem_bytes) {
+  (void)G;
+  return (size_t)combine_smem(hd, H, n_split, elem_bytes).total * sizeof(float);
 }
 
 cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
@@ -280,18 +307,28 @@ cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
-  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.G, a.n_split);
-  dim3 grid(a.Hkv, a.B);
+  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.G, a.n_split, dt == LR_BF16 ? 2 : 4);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(ceil_div(a.hd, CJ), a.Hkv * a.G, a.B);
+  cfg.blockDim = dim3(CT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e;
   if (dt == LR_BF16) {
     e = cudaFuncSetAttribute(decode_combine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<__nv_bfloat16><<<grid, CT, smem, st>>>(a);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<__nv_bfloat16>, a);
   } else {
     e = cudaFuncSetAttribute(decode_combine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_combine_kernel<float><<<grid, CT, smem, st>>>(a);
+    e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<float>, a);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -580,9 +580,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
   const int s = blockIdx.x, hp = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H, nh = a.H / 128, nk = a.r / kChunk, nw = 2 * nh;
-  const int n_tiles = tile_count(a, b, hp);
-  const int t_begin = (int)((long long)s * n_tiles / a.n_split);
-  const int t_end = (int)((long long)(s + 1) * n_tiles / a.n_split);
   const int ha = 2 * hp;  // first KV head of the pair
 
   // ---------------------------------------------------------------- setup
@@ -636,6 +633,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // The setup above overlaps the end of the prep grid (programmatic dependent launch);
+  // its outputs (schedule, Qhat, fp16 W1) are read only after this wait.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int n_tiles = tile_count(a, b, hp);
+  const int t_begin = (int)((long long)s * n_tiles / a.n_split);
+  const int t_end = (int)((long long)(s + 1) * n_tiles / a.n_split);
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
@@ -794,6 +797,7 @@ template <int MG>
 __global__ void __launch_bounds__(256) decode_tc_prep_kernel(TcArgs a, int n_w1, int n_q, const int* blocks,
                                                              int n_sel) {
   const int bid = blockIdx.x, tid = threadIdx.x;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // inputs come from the kernels before this one
   if (bid < n_w1) {
     const size_t per_seq = (size_t)a.Hkv * a.H * kHd;
     const size_t n = (size_t)a.w1_seqs * per_seq;
@@ -896,13 +900,27 @@ cudaError_t launch_mg(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap&
   const int n_w1 = (int)((n_w1_vec + 255) / 256 < 512 ? (n_w1_vec + 255) / 256 : 512);
   const int n_q = ((a.r + 63) / 64) * a.Hkv * a.B;
   const int n_s = a.sched ? a.n_hp * a.B : 0;
-  decode_tc_prep_kernel<MG><<<n_w1 + n_q + n_s, 256, 0, st>>>(a, n_w1, n_q, blocks, n_sel);
-  cudaError_t e = cudaGetLastError();
+  // both kernels may be launched while the previous grid drains; each waits for it
+  // (griddepcontrol.wait) before it reads anything that grid writes
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(n_w1 + n_q + n_s);
+  cfg.blockDim = dim3(256);
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_prep_kernel<MG>, a, n_w1, n_q, blocks, n_sel);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(decode_tc_kernel<MG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Layout<MG>::kSmemBytes);
   if (e != cudaSuccess) return e;
-  decode_tc_kernel<MG><<<dim3(a.n_split, a.n_hp, a.B), kThreads, Layout<MG>::kSmemBytes, st>>>(mA, mB, mQ, mW1, a);
+  cfg.gridDim = dim3(a.n_split, a.n_hp, a.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = Layout<MG>::kSmemBytes;
+  e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MG>, mA, mB, mQ, mW1, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
