@@ -72,6 +72,7 @@ typedef enum lr_dtype { LR_F32 = 0, LR_BF16 = 1 } lr_dtype;
 #define LR_DEVERR_RES_ORDER 8   /* residual indices not strictly ascending */
 #define LR_DEVERR_PTR 16        /* a residual block pointer out of [0, k] or decreasing */
 #define LR_DEVERR_TIMEOUT 32    /* a kernel gave up waiting on its own pipeline (its output is invalid) */
+#define LR_DEVERR_LAUNCH 64     /* a kernel found its shared memory misaligned and did not run (output invalid) */
 
 typedef struct lr_cache_shape {
   int32_t batch;      /* B >= 0 */

@@ -11,11 +11,12 @@ namespace lr {
 struct DecodeArgs;
 struct PackArgs;
 
-enum class DecodePath { General = 0, Tensor = 1 };
+enum class DecodePath { General = 0, Tensor = 1, Pair = 2 };
 
 struct DecodePlan {
   DecodePath path;
-  int n_split;       // token splits per (sequence, KV head) (general) or per sequence (tensor)
+  int n_split;       // split partials per query head
+  int n_pairs;       // pair path: CTA pairs per (sequence, KV head)
   int part_stride;   // floats per split partial
   size_t part_off;   // byte offset of the partials in the workspace
   size_t sched_off;  // byte offset of the tensor path's block schedule
@@ -32,6 +33,7 @@ struct PackPlan {
 };
 
 bool decode_tc_supported(const lr_cache_shape& s, int n_q_heads);
+bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads);
 DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);
 PackPlan plan_pack(const lr_cache_shape& s, int k);
 

@@ -20,6 +20,7 @@ LR_OK, LR_ERR_INVALID_ARG, LR_ERR_UNSUPPORTED, LR_ERR_WORKSPACE, LR_ERR_CUDA, LR
 LR_F32, LR_BF16 = 0, 1
 LR_BLOCK_TOKENS = 64
 LR_DEVERR_BLOCK_RANGE, LR_DEVERR_BLOCK_ORDER, LR_DEVERR_RES_RANGE, LR_DEVERR_RES_ORDER, LR_DEVERR_PTR = 1, 2, 4, 8, 16
+LR_DEVERR_TIMEOUT, LR_DEVERR_LAUNCH = 32, 64
 
 _DT = {torch.float32: LR_F32, torch.bfloat16: LR_BF16}
 
