@@ -216,11 +216,32 @@ def build_cache(w: synth.Workload, lr, seed_offset: int = 0):
 
 
 def decode_launches_per_step(w: synth.Workload, n_sel: int) -> int:
-    """Kernels one lr_decode_attn call launches (tensor-core path: prep, main kernel, combine;
-    general path: main kernel, combine)."""
+    """Kernels one lr_decode_attn call launches (tensor-core paths: prep, main kernel,
+    combine; general path: main kernel, combine)."""
     tc = (w.dtype == "bf16" and w.head_dim == 128 and w.hidden in (128, 256) and w.rank % 64 == 0
-          and w.n_kv_heads % 2 == 0 and w.q_per_kv <= 8 and w.T > 0)
+          and w.q_per_kv <= 8 and w.T > 0)
     return 3 if tc else 2
+
+
+# DRAM bytes (read + write) per launch of the decode kernel, from one ncu capture of the
+# kernel source whose SHA-256 prefix is given (profiles/launches_pair_path_*.md). Reported
+# as roofline.traffic only while the source is unchanged; otherwise traffic is null.
+NCU_TRAFFIC = {
+    "mistral_group_32k": ("0f7b02d23a7ebf44", 76.96e6 + 0.56e6),
+}
+
+
+def measured_traffic(workload: str):
+    entry = NCU_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    path = os.path.join(ROOT, "long_context_decode_lr_b200", "csrc", "decode_pair.cu")
+    try:
+        with open(path, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return entry[1] if digest == entry[0] else None
 
 
 def clone_cache(c, lr):
@@ -326,7 +347,7 @@ def run_lowram(args, world, rank):
                    "parallelism": f"dp{world}" if world > 1 else "single"},
         "us_per_layer": ms_step * 1e3, "model_32_layers_ms": ms_step * 32,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": measured_traffic(w.name),
                      "kernel": "lr_decode_attn (split kernel + combine; event time covers both)",
                      "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
                      "peak_source": f"{pk_kind} ({'sustained' if tpeak == pk.get('bf16_tflops_sustained') else 'burst'} bf16)"},
