@@ -133,3 +133,18 @@ def test_full_size(name, sel):
     got, ref, code = _run(p, layer=layer)
     assert code == 0
     H.assert_attention_close(got, ref)
+
+
+# The library picks the CTA-pair kernel for bf16 / head_dim 128 caches. The single-CTA
+# tensor-core kernel and the CUDA-core kernel stay available as fallbacks; forcing each one
+# (LOWRAM_DECODE_PATH) keeps them under the same parity bar.
+@pytest.mark.parametrize("path", ["tensor", "general"])
+@pytest.mark.parametrize("name", ["ragged_full", "ragged_sel5", "gqa8_b2", "batch2_sel"])
+def test_fallback_paths(name, path, monkeypatch):
+    monkeypatch.setenv("LOWRAM_DECODE_PATH", path)
+    c = CASES[name]
+    w = H.small(**c["w"])
+    p = H.packed_problem(w, k=c.get("k"), with_b2=c.get("b2", False), sel=c.get("sel"))
+    got, ref, code = _run(p, use_ptr=c.get("ptr", True), scale=c.get("scale", 0.0))
+    assert code == 0
+    H.assert_attention_close(got, ref)
