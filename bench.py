@@ -136,16 +136,23 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU (torchrun env). NCCL on GPUs; gloo exercises the same host
+    logic on CPU. Returns (world, rank, local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
@@ -158,12 +165,25 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Device time of a multi-rank run: the slowest rank's."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Weak scaling: every rank decodes its own sequences, drawn from its own seed."""
+    return rank
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_step: float) -> float:
+    """Whole-job throughput: the context tokens all ranks processed in one step, over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_step * 1e-3)
 
 
 # ----------------------------------------------------------------------------- cache
@@ -260,7 +280,7 @@ def run_lowram(args, world, rank):
     lr.library()
     w = synth.WORKLOADS[args.workload]
     n_sel = w.n_sel
-    c0, shape, _, pack = build_cache(w, lr, seed_offset=rank)
+    c0, shape, _, pack = build_cache(w, lr, seed_offset=rank_seed_offset(rank))
     per_copy = sum(t.numel() * t.element_size() for t in c0.values() if isinstance(t, torch.Tensor))
     n_copies = max(2, math.ceil(2.2 * L2_BYTES / max(per_copy, 1)))
     copies = [clone_cache(c0, lr) for _ in range(n_copies)]
@@ -333,8 +353,7 @@ def run_lowram(args, world, rank):
         achieved, peak, unit = flops / s_step / 1e12, tpeak, "TFLOP/s"
     else:
         achieved, peak, unit = bytes_ / s_step / 1e9, pk["hbm_gbs"], "GB/s"
-    tokens = w.batch * w.T * world
-    value = tokens / s_step
+    value = job_tokens_per_s(w.batch * w.T, world, ms_step)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -352,7 +371,7 @@ def run_lowram(args, world, rank):
                      "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
                      "peak_source": f"{pk_kind} ({'sustained' if tpeak == pk.get('bf16_tflops_sustained') else 'burst'} bf16)"},
         "roofline_pct": 100.0 * max(t_tensor, t_hbm) / s_step,
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(w.batch * w.T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "d2h_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "ms_per_step": e2e_ms},
