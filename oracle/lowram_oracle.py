@@ -192,7 +192,8 @@ def selected_tokens(T: int, blocks: Optional[Sequence[int]], block: int = BLOCK)
 
 
 def decode_sequence(q, A, Bt, W_lin, W1, b1, W2, b2, layer: int, res_idx, res_val,
-                    blocks, scale: float, n_kv_heads: int, head_dim: int) -> np.ndarray:
+                    blocks, scale: float, n_kv_heads: int, head_dim: int,
+                    tail_K=None, tail_V=None) -> np.ndarray:
     """One decode step of one layer for one sequence: o [Hq, hd].
 
     For KV head h: gather the attended tokens (all, or the selected blocks:
@@ -202,22 +203,34 @@ def decode_sequence(q, A, Bt, W_lin, W1, b1, W2, b2, layer: int, res_idx, res_va
     h*G .. h*G+G-1 with max-subtracted exponentials. Predictor arrays are
     indexed [L, Hkv, ...]; res_idx [L, Hkv, k]; res_val [L, Hkv, k, hd];
     blocks is None (all tokens) or a per-KV-head sequence of block ids.
+
+    tail_K, tail_V [Hkv, n_tail, hd] (optional): tokens generated after the cache was
+    packed, kept exactly (explainer, paragraph on prefill and decode costs: newly
+    generated tokens are stored exactly). They join the same softmax with their own
+    keys and values, whatever the block selection.
     """
     q = np.asarray(q, np.float64)
     Hq = q.shape[0]
     G = Hq // n_kv_heads
     T = A.shape[0]
+    n_tail = 0 if tail_K is None else np.asarray(tail_K).shape[1]
     o = np.zeros((Hq, head_dim), np.float64)
     for h in range(n_kv_heads):
         S = selected_tokens(T, None if blocks is None else blocks[h])
-        if S.size == 0:
+        kt = np.zeros((0, head_dim), np.float64)
+        v = np.zeros((0, head_dim), np.float64)
+        if S.size:
+            kt = reconstruct_keys(np.asarray(A, np.float64)[S], key_slice(Bt, layer, h, n_kv_heads, head_dim))
+            v = predict_values(kt, W_lin[layer, h], W1[layer, h], b1[layer, h], W2[layer, h],
+                               None if b2 is None else b2[layer, h])
+            r_full = np.zeros((T, head_dim), np.float64)
+            r_full[np.asarray(res_idx[layer, h], np.int64)] = np.asarray(res_val[layer, h], np.float64)
+            v = v + r_full[S]
+        if n_tail:
+            kt = np.concatenate([kt, np.asarray(tail_K[h], np.float64)])
+            v = np.concatenate([v, np.asarray(tail_V[h], np.float64)])
+        if kt.shape[0] == 0:
             continue
-        kt = reconstruct_keys(np.asarray(A, np.float64)[S], key_slice(Bt, layer, h, n_kv_heads, head_dim))
-        v = predict_values(kt, W_lin[layer, h], W1[layer, h], b1[layer, h], W2[layer, h],
-                           None if b2 is None else b2[layer, h])
-        r_full = np.zeros((T, head_dim), np.float64)
-        r_full[np.asarray(res_idx[layer, h], np.int64)] = np.asarray(res_val[layer, h], np.float64)
-        v = v + r_full[S]
         for g in range(G):
             hq = h * G + g
             s = (kt @ q[hq]) * scale

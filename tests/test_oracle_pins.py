@@ -284,3 +284,52 @@ def test_dense_cache_bytes():
     g = _gold("dense_cache_size.json")
     b = orc.dense_cache_bytes_per_token(g["n_layers"], g["n_kv_heads"], g["head_dim"], g["elem_bytes"])
     assert round(b / 1000, 2) == g["kb_per_token_printed"]
+
+
+@pytest.mark.parametrize("selective", [False, True])
+def test_tail_joins_the_softmax_as_dense_tokens(selective):
+    """Exact recent-token tail: with k = T residuals and a full-rank key factor the cache is
+    exact, so decode with a tail equals dense attention over the attended cache tokens
+    followed by the tail tokens (explainer: newly generated tokens are stored exactly)."""
+    rng = np.random.default_rng(71 + selective)
+    L, Hkv, G, hd, T, n_tail = 1, 2, 2, 16, 200, 5
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])
+    packed = orc.pack_sequence(K_group, V, Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"],
+                               pred["b2"], T, "f64", Hkv, hd)
+    tail_K = rng.standard_normal((Hkv, n_tail, hd))
+    tail_V = rng.standard_normal((Hkv, n_tail, hd))
+    blocks = [[1], [0, 2, 3]] if selective else None
+    q = rng.standard_normal((Hkv * G, hd))
+    o = orc.decode_sequence(q, packed["A"], Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"], pred["b2"],
+                            0, packed["idx"], packed["val"], blocks, 0.3, Hkv, hd, tail_K, tail_V)
+    for hq in range(Hkv * G):
+        h = hq // G
+        S = orc.selected_tokens(T, None if blocks is None else blocks[h])
+        K = np.concatenate([K_group[S, h * hd:(h + 1) * hd], tail_K[h]])
+        Vh = np.concatenate([V[0][S, h], tail_V[h]])
+        np.testing.assert_allclose(o[hq], orc.dense_attention(q[hq], K, Vh, 0.3), rtol=1e-10, atol=1e-10)
+
+
+def test_tail_alone_and_tail_order():
+    """A single tail token with nothing else attended is the output itself (softmax over one
+    element); the tail's order does not matter."""
+    rng = np.random.default_rng(5)
+    L, Hkv, G, hd, T = 1, 2, 4, 16, 150
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])[:, :24]
+    packed = orc.pack_sequence(K_group, V, Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"],
+                               pred["b2"], 10, "bf16", Hkv, hd)
+    args = (packed["A"], Bt, pred["W_lin"], pred["W1"], pred["b1"], pred["W2"], pred["b2"], 0,
+            packed["idx"], packed["val"])
+    q = rng.standard_normal((Hkv * G, hd))
+    tK, tV = rng.standard_normal((Hkv, 1, hd)), rng.standard_normal((Hkv, 1, hd))
+    only = orc.decode_sequence(q, *args, [[], []], 0.25, Hkv, hd, tK, tV)
+    for hq in range(Hkv * G):
+        np.testing.assert_array_equal(only[hq], tV[hq // G, 0])
+    tK, tV = rng.standard_normal((Hkv, 6, hd)), rng.standard_normal((Hkv, 6, hd))
+    perm = rng.permutation(6)
+    a = orc.decode_sequence(q, *args, None, 0.25, Hkv, hd, tK, tV)
+    b = orc.decode_sequence(q, *args, None, 0.25, Hkv, hd, tK[:, perm], tV[:, perm])
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    assert not np.allclose(a, orc.decode_sequence(q, *args, None, 0.25, Hkv, hd))
