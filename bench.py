@@ -52,7 +52,7 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_work(w: synth.Workload, n_sel: int):
+def algorithmic_work(w: synth.Workload, n_sel: int, n_tail: int = 0):
     """(tensor FLOPs, HBM bytes) one decode step of one layer must do at minimum.
 
     Per attended token and KV head: the key rebuild A.B_l^h (2 r hd FLOPs) and the
@@ -60,7 +60,8 @@ def algorithmic_work(w: synth.Workload, n_sel: int):
     query head after the softmax sums, so they do not scale with tokens. Bytes: the
     A rows of the attended tokens (each row once), the layer's basis slice and
     predictors per sequence, the residual rows and indices of attended tokens, the
-    block lists and the query/output.
+    block lists and the query/output; an exact tail adds its keys and values (read once)
+    and 4 hd FLOPs per query head and tail token.
     """
     e = 2
     B, T, r, hd, H, Hkv, Hq = w.batch, w.T, w.rank, w.head_dim, w.hidden, w.n_kv_heads, w.n_q_heads
@@ -80,7 +81,9 @@ def algorithmic_work(w: synth.Workload, n_sel: int):
                   + Hkv * w.k * res_frac * (hd * e + 4)           # residual rows + indices
                   + Hkv * (w.nblk + 1) * 4                        # block pointers
                   + Hkv * n_sel * 4                               # block lists
-                  + 2 * Hq * hd * e)                              # q and o
+                  + 2 * Hq * hd * e                               # q and o
+                  + 2 * Hkv * n_tail * hd * e)                    # exact tail keys and values
+    flops += B * Hq * n_tail * 4 * hd
     return float(flops), float(bytes_)
 
 
@@ -294,12 +297,26 @@ def run_lowram(args, world, rank):
     stream = torch.cuda.current_stream()
     k = w.k
 
+    n_tail = args.tail
+    tails = None
+    if n_tail:
+        mw = synth.model_weights(w)
+        tails = []
+        for l in range(w.n_layers):
+            Kt, Vt = synth.tail_tokens(w, mw, l, n_tail)
+            tails.append(tuple(synth.to_storage(x, w.dtype)[0].cuda().contiguous() for x in (Kt, Vt)))
+
     def step(i, q=None, o=None):
         c = copies[i % n_copies]
         layer = (i // n_copies) % w.n_layers
-        lr.lr_decode_attn(shape, layer, w.n_q_heads, c["q"][layer] if q is None else q, c["A"], c["Bt"],
-                          c["pred"], c["idx"], c["val"], c["ptr"], k, blocks, n_sel, 0.0,
-                          outs[i & 1] if o is None else o, ws, stream)
+        qq, oo = c["q"][layer] if q is None else q, outs[i & 1] if o is None else o
+        if n_tail:
+            lr.lr_decode_attn_tail(shape, layer, w.n_q_heads, qq, c["A"], c["Bt"], c["pred"], c["idx"], c["val"],
+                                   c["ptr"], k, blocks, n_sel, tails[layer][0], tails[layer][1], n_tail, 0.0, oo,
+                                   ws, stream)
+        else:
+            lr.lr_decode_attn(shape, layer, w.n_q_heads, qq, c["A"], c["Bt"], c["pred"], c["idx"], c["val"],
+                              c["ptr"], k, blocks, n_sel, 0.0, oo, ws, stream)
 
     for i in range(args.warmup):
         step(i)
@@ -341,7 +358,7 @@ def run_lowram(args, world, rank):
 
     if rank != 0:
         return None
-    flops, bytes_ = algorithmic_work(w, n_sel)
+    flops, bytes_ = algorithmic_work(w, n_sel, n_tail)
     pk, pk_kind = peaks()
     timed_s = ms_total * 1e-3
     tpeak = pk["bf16_tflops_sustained"] if timed_s > 2.0 else pk["bf16_tflops"]
@@ -353,14 +370,17 @@ def run_lowram(args, world, rank):
         achieved, peak, unit = flops / s_step / 1e12, tpeak, "TFLOP/s"
     else:
         achieved, peak, unit = bytes_ / s_step / 1e9, pk["hbm_gbs"], "GB/s"
-    value = job_tokens_per_s(w.batch * w.T, world, ms_step)
+    ctx = w.batch * (w.T + n_tail)  # context tokens attended per step: the cache plus the exact tail
+    value = job_tokens_per_s(ctx, world, ms_step)
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "description": w.description, "batch_per_gpu": w.batch,
                    "context": w.T, "mode": "selective" if n_sel else "full", "n_sel": n_sel,
-                   "residual_pct": w.res_pct, "step": "one lr_decode_attn call (one layer)",
+                   "residual_pct": w.res_pct, "tail": n_tail,
+                   "step": "one lr_decode_attn call (one layer)" if not n_tail else
+                           f"one lr_decode_attn_tail call (one layer, {n_tail} exact tail tokens per KV head)",
                    "l2": f"inputs rotate over {n_copies} device copies of the cache "
                          f"({n_copies * per_copy / 2**20:.0f} MB > L2)",
                    "parallelism": f"dp{world}" if world > 1 else "single"},
@@ -371,7 +391,7 @@ def run_lowram(args, world, rank):
                      "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
                      "peak_source": f"{pk_kind} ({'sustained' if tpeak == pk.get('bf16_tflops_sustained') else 'burst'} bf16)"},
         "roofline_pct": 100.0 * max(t_tensor, t_hbm) / s_step,
-        "e2e": {"value": job_tokens_per_s(w.batch * w.T, world, e2e_ms), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(ctx, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "d2h_bytes_per_step": w.batch * w.n_q_heads * w.head_dim * (2 if dt == torch.bfloat16 else 4),
                 "ms_per_step": e2e_ms},
@@ -465,6 +485,8 @@ def main():
     ap.add_argument("--workload", default="mistral_group_32k", choices=synth.names())
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--tail", type=int, default=0,
+                    help="exact recent tokens per (sequence, KV head) decoded with the cache (lr_decode_attn_tail)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -170,6 +170,35 @@ lr_status lr_decode_attn(const lr_cache_shape* shape, int32_t layer, int32_t n_q
                          const int32_t* block_list, int32_t n_sel, float scale, void* o,
                          void* ws, size_t ws_bytes, lr_stream_t stream);
 
+/* Largest exact tail lr_decode_attn_tail accepts. */
+#define LR_MAX_TAIL 4096
+
+/*
+ * lr_decode_attn_tail -- lr_decode_attn with an exact recent-token tail.
+ *
+ * Tokens generated after the cache was packed are kept exactly until the cache is packed
+ * again (explainer, paragraph on prefill and decode costs: newly generated tokens are
+ * stored exactly). They join the same softmax with their own keys and values:
+ *   o[b, hq] = sum_{t in S + tail} softmax_t(scale * q[b, hq] . key_t) value_t,
+ * where a tail token i of KV head h has key tail_K[b, h, i] and value tail_V[b, h, i]
+ * (this layer's), and S is the compressed set of lr_decode_attn.
+ *
+ * Inputs:  those of lr_decode_attn, plus tail_K, tail_V [B, Hkv, n_tail, hd] in the cache
+ *          dtype (caller-owned device memory, this layer's slices), 0 <= n_tail <=
+ *          LR_MAX_TAIL; tail_K / tail_V may be NULL when n_tail == 0, which makes the call
+ *          lr_decode_attn. The tail is attended whatever block_list selects; T may be 0.
+ * Output:  o [B, Hq, hd]. Workspace: lr_decode_workspace_bytes, as for lr_decode_attn.
+ * Errors:  as lr_decode_attn; n_tail outside [0, LR_MAX_TAIL] or a NULL tail with
+ *          n_tail > 0 return LR_ERR_INVALID_ARG before any launch.
+ */
+lr_status lr_decode_attn_tail(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
+                              const void* q, const void* A, const void* Bt,
+                              const lr_predictor* predictor, const int32_t* res_idx,
+                              const void* res_val, const int32_t* res_blk_ptr, int32_t k,
+                              const int32_t* block_list, int32_t n_sel, const void* tail_K,
+                              const void* tail_V, int32_t n_tail, float scale, void* o,
+                              void* ws, size_t ws_bytes, lr_stream_t stream);
+
 /* ------------------------------------------------------------------ single steps */
 
 /* Workspace bytes lr_topk_tokens needs. */

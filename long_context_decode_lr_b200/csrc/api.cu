@@ -121,11 +121,14 @@ size_t lr_decode_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads, int
   return lr::plan_decode(*s, n_q_heads, n_sel, current_sm_count()).ws_bytes;
 }
 
-lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
-                         const void* A, const void* Bt, const lr_predictor* pred,
-                         const int32_t* res_idx, const void* res_val, const int32_t* res_blk_ptr,
-                         int32_t k, const int32_t* block_list, int32_t n_sel, float scale, void* o,
-                         void* ws, size_t ws_bytes, lr_stream_t stream) {
+}  // extern "C"
+
+namespace {
+lr_status decode_impl(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q, const void* A,
+                      const void* Bt, const lr_predictor* pred, const int32_t* res_idx, const void* res_val,
+                      const int32_t* res_blk_ptr, int32_t k, const int32_t* block_list, int32_t n_sel,
+                      const void* tail_K, const void* tail_V, int32_t n_tail, float scale, void* o, void* ws,
+                      size_t ws_bytes, lr_stream_t stream) {
   lr_status st = check_shape(s);
   if (st != LR_OK) return st;
   if (layer < 0 || layer >= s->n_layers) return fail(LR_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, s->n_layers);
@@ -146,6 +149,11 @@ lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_hea
   }
   CHECK_OPT_PTR(res_blk_ptr, "res_blk_ptr");
   CHECK_OPT_PTR(block_list, "block_list");
+  if (n_tail < 0 || n_tail > LR_MAX_TAIL) return fail(LR_ERR_INVALID_ARG, "n_tail=%d outside [0, %d]", n_tail, LR_MAX_TAIL);
+  if (n_tail > 0) {
+    CHECK_PTR(tail_K, "tail_K");
+    CHECK_PTR(tail_V, "tail_V");
+  }
   const lr::DecodePlan plan = lr::plan_decode(*s, n_q_heads, n_sel, current_sm_count());
   if ((st = check_ws(ws, ws_bytes, plan.ws_bytes)) != LR_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
@@ -164,6 +172,9 @@ lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_hea
   a.res_idx = k ? res_idx : nullptr; a.res_val = k ? res_val : nullptr;
   a.res_ptr = k ? res_blk_ptr : nullptr;
   a.blocks = block_list;
+  a.tail_K = n_tail ? tail_K : nullptr;
+  a.tail_V = n_tail ? tail_V : nullptr;
+  a.n_tail = n_tail;
   a.o = o;
   a.err = (int*)ws;
   a.partials = (float*)((char*)ws + plan.part_off);
@@ -171,6 +182,28 @@ lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_hea
   a.part_stride = plan.part_stride;
   if ((e = lr::launch_decode(a, plan, s->dtype, cs)) != cudaSuccess) return cuda_fail(e, "decode launch");
   return LR_OK;
+}
+}  // namespace
+
+extern "C" {
+
+lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
+                         const void* A, const void* Bt, const lr_predictor* pred,
+                         const int32_t* res_idx, const void* res_val, const int32_t* res_blk_ptr,
+                         int32_t k, const int32_t* block_list, int32_t n_sel, float scale, void* o,
+                         void* ws, size_t ws_bytes, lr_stream_t stream) {
+  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, res_val, res_blk_ptr, k, block_list, n_sel,
+                     nullptr, nullptr, 0, scale, o, ws, ws_bytes, stream);
+}
+
+lr_status lr_decode_attn_tail(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
+                              const void* A, const void* Bt, const lr_predictor* pred,
+                              const int32_t* res_idx, const void* res_val, const int32_t* res_blk_ptr,
+                              int32_t k, const int32_t* block_list, int32_t n_sel, const void* tail_K,
+                              const void* tail_V, int32_t n_tail, float scale, void* o, void* ws,
+                              size_t ws_bytes, lr_stream_t stream) {
+  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, res_val, res_blk_ptr, k, block_list, n_sel,
+                     tail_K, tail_V, n_tail, scale, o, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ pack

@@ -161,7 +161,11 @@ __global__ void __launch_bounds__(NT) decode_general_kernel(DecodeArgs a) {
 }
 
 // Merge the split partials of one query head and apply the linear maps once:
-// o = (acc_k W_lin^T + acc_g W2^T + acc_r) / l + b2. One block per (chunk of CJ output
+// o = (acc_k W_lin^T + acc_g W2^T + acc_r + l_c b2 + sum_tail w_t v_t) / (l_c + l_tail),
+// where the exact tail tokens (newly generated, stored exactly) join the softmax here with
+// their own keys and values, all weights taken relative to one maximum over the splits
+// and the tail; without a tail this is (acc_k W_lin^T + acc_g W2^T + acc_r) / l + b2.
+// One block per (chunk of CJ output
 // columns, query head, sequence), so that even a single sequence spreads over many SMs;
 // every block of a head re-merges acc_k and acc_g (hd + H floats per split, read from
 // L2) and only its own CJ columns of acc_r. The kernel may start while the split kernel
@@ -175,10 +179,10 @@ constexpr int kMaxChunk = 8; // split chunks per merged entry
 
 struct CombineSmem {
   int n_ch, cs, n_acc, w_floats;
-  int off_ml, off_w, off_red, off_acc, total;  // in floats
+  int off_ml, off_w, off_red, off_acc, off_tail, off_q, off_tred, total;  // in floats
 };
 
-__host__ __device__ inline CombineSmem combine_smem(int hd, int H, int S, int elem_bytes) {
+__host__ __device__ inline CombineSmem combine_smem(int hd, int H, int S, int elem_bytes, int n_tail) {
   CombineSmem c;
   c.n_ch = ceil_div(S, 8) < kMaxChunk ? ceil_div(S, 8) : kMaxChunk;
   c.cs = ceil_div(S, c.n_ch);
@@ -188,30 +192,53 @@ __host__ __device__ inline CombineSmem combine_smem(int hd, int H, int S, int el
   c.off_ml = c.w_floats;
   c.off_red = c.off_ml + 2 * S;
   c.off_acc = c.off_red + c.n_ch * c.n_acc;
-  c.total = c.off_acc + c.n_acc;
+  c.off_tail = c.off_acc + c.n_acc;                    // [n_tail] tail scores, then weights
+  c.off_q = c.off_tail + n_tail;                       // [hd] the query
+  c.off_tred = c.off_q + (n_tail ? hd : 0);            // [warps][CJ] tail value sums
+  c.total = c.off_tred + (n_tail ? (CT / 32) * CJ : 0);
   return c;
 }
 
 template <typename T>
 __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
   extern __shared__ float sm[];
-  __shared__ float s_m, s_inv_l, s_b2[CJ];
+  __shared__ float s_lc, s_lt, s_b2[CJ];
   const int jc = blockIdx.x, qh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int hd = a.hd, H = a.H, Hq = a.Hkv * a.G, S = a.n_split;
+  const int hd = a.hd, H = a.H, Hq = a.Hkv * a.G, S = a.n_split, nt = a.n_tail;
   const int j0 = jc * CJ, nj = min(CJ, hd - j0);
-  const CombineSmem L = combine_smem(hd, H, S, (int)sizeof(T));
+  const CombineSmem L = combine_smem(hd, H, S, (int)sizeof(T), nt);
   T* wl_s = reinterpret_cast<T*>(sm + L.off_w);  // [nj][hd]
   T* w2_s = wl_s + CJ * hd;                      // [nj][H]
   float* mls = sm + L.off_ml;                    // [S] maxima, then [S] sums
   float* red = sm + L.off_red;                   // [n_ch][n_acc]
   float* acc = sm + L.off_acc;                   // [hd + H + nj]: merged sum p k~, sum p g, own columns of sum p r
+  float* ts = sm + L.off_tail;                   // [nt] exact tail tokens: scores, then softmax weights
+  float* tred = sm + L.off_tred;                 // [warps][CJ] tail value sums per warp
 
   // weight rows are inputs of the call, independent of the split kernel
   const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, qh / a.G);
   for (int i = tid; i < nj * hd; i += CT) wl_s[i] = P.W_lin[(size_t)j0 * hd + i];
   for (int i = tid; i < nj * H; i += CT) w2_s[i] = P.W2[(size_t)j0 * H + i];
   if (tid < nj) s_b2[tid] = P.b2 ? to_f32(P.b2[j0 + tid]) : 0.f;
+  // scores of the exact tail tokens (inputs of the call as well): scale q . key_t
+  const int h = qh / a.G;
+  if (nt > 0) {
+    float* qv = sm + L.off_q;
+    const T* qp = (const T*)a.q + ((size_t)b * Hq + qh) * hd;
+    for (int d = tid; d < hd; d += CT) qv[d] = to_f32(qp[d]);
+    __syncthreads();
+    const T* kt = (const T*)a.tail_K + ((size_t)b * a.Hkv + h) * nt * hd;
+    for (int t = tid; t < nt; t += CT) {
+      const T* kr = kt + (size_t)t * hd;
+      float s0 = 0.f, s1 = 0.f;
+      for (int d = 0; d < hd; d += 2) {
+        s0 = fmaf(qv[d], to_f32(kr[d]), s0);
+        s1 = fmaf(qv[d + 1], to_f32(kr[d + 1]), s1);
+      }
+      ts[t] = (s0 + s1) * a.scale;
+    }
+  }
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const float* part = a.partials + ((size_t)b * Hq + qh) * S * a.part_stride;
@@ -220,24 +247,38 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
     mls[S + s] = part[(size_t)s * a.part_stride + 1];
   }
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0) {  // one max over the splits and the tail; weights relative to it
     float m = -CUDART_INF_F;
     for (int s = lane; s < S; s += 32) m = fmaxf(m, mls[s]);
+    for (int t = lane; t < nt; t += 32) m = fmaxf(m, ts[t]);
     m = warp_max(m);
-    float l = 0.f;
+    float lc = 0.f, lt = 0.f;
     for (int s = lane; s < S; s += 32) {
       const float ms = mls[s];
       const float wgt = (m == -CUDART_INF_F || ms == -CUDART_INF_F) ? 0.f : __expf(ms - m);
       mls[s] = wgt;
-      l = fmaf(wgt, mls[S + s], l);
+      lc = fmaf(wgt, mls[S + s], lc);
     }
-    l = warp_sum(l);
+    for (int t = lane; t < nt; t += 32) {
+      const float wgt = m == -CUDART_INF_F ? 0.f : __expf(ts[t] - m);
+      ts[t] = wgt;
+      lt += wgt;
+    }
+    lc = warp_sum(lc);
+    lt = warp_sum(lt);
     if (lane == 0) {
-      s_m = m;
-      s_inv_l = l > 0.f ? 1.f / l : 0.f;
+      s_lc = lc;
+      s_lt = lt;
     }
   }
   __syncthreads();
+  if (nt > 0) {  // tail values weighted by their softmax weights, this block's columns
+    const T* vt = (const T*)a.tail_V + ((size_t)b * a.Hkv + h) * nt * hd + j0;
+    float av = 0.f;
+    if (lane < nj)
+      for (int t = warp; t < nt; t += CT / 32) av = fmaf(ts[t], to_f32(vt[(size_t)t * hd + lane]), av);
+    tred[warp * CJ + lane] = av;
+  }
   const int n_acc = hd + H + nj;
   for (int it = tid; it < L.n_ch * n_acc; it += CT) {
     const int c = it / n_acc, x = it % n_acc;
@@ -264,7 +305,7 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
   }
   __syncthreads();
   T* o = (T*)a.o + ((size_t)b * Hq + qh) * hd;
-  const float m = s_m, inv_l = s_inv_l;
+  const float lc = s_lc, lsum = s_lc + s_lt;
   for (int jj = warp; jj < nj; jj += CT / 32) {
     const T* wl = wl_s + jj * hd;
     const T* w2 = w2_s + jj * H;
@@ -273,7 +314,9 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
     for (int c = lane; c < H; c += 32) y1 = fmaf(acc[hd + c], to_f32(w2[c]), y1);
     const float y = warp_sum(y0 + y1);
     if (lane == 0) {
-      const float out = m == -CUDART_INF_F ? 0.f : (y + acc[hd + H + jj]) * inv_l + s_b2[jj];
+      float tv = 0.f;
+      for (int w = 0; w < (nt > 0 ? CT / 32 : 0); ++w) tv += tred[w * CJ + jj];
+      const float out = lsum > 0.f ? (y + acc[hd + H + jj] + lc * s_b2[jj] + tv) / lsum : 0.f;
       o[j0 + jj] = from_f32<T>(out);
     }
   }
@@ -285,9 +328,9 @@ size_t decode_general_smem_bytes(int hd, int H, int G) {
   return (size_t)decode_smem_plan(hd, H, G).total * sizeof(float);
 }
 
-size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split, int elem_bytes) {
+size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split, int elem_bytes, int n_tail) {
   (void)G;
-  return (size_t)combine_smem(hd, H, n_split, elem_bytes).total * sizeof(float);
+  return (size_t)combine_smem(hd, H, n_split, elem_bytes, n_tail).total * sizeof(float);
 }
 
 cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
@@ -307,7 +350,7 @@ cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t
 }
 
 cudaError_t launch_decode_combine(const DecodeArgs& a, lr_dtype dt, cudaStream_t st) {
-  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.G, a.n_split, dt == LR_BF16 ? 2 : 4);
+  const size_t smem = decode_combine_smem_bytes(a.hd, a.H, a.G, a.n_split, dt == LR_BF16 ? 2 : 4, a.n_tail);
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(ceil_div(a.hd, CJ), a.Hkv * a.G, a.B);
   cfg.blockDim = dim3(CT);

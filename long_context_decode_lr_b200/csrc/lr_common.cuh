@@ -63,6 +63,9 @@ struct DecodeArgs {
   const void* res_val;  // [B, L, Hkv, k, hd]
   const int* res_ptr;   // [B, L, Hkv, nblk + 1] or null
   const int* blocks;    // [B, Hkv, n_sel] or null
+  const void* tail_K;   // [B, Hkv, n_tail, hd] exact recent tokens, or null
+  const void* tail_V;   // [B, Hkv, n_tail, hd]
+  int n_tail;
   void* o;              // [B, Hq, hd]
   float* partials;      // [B, Hq, n_split, part_stride]
   int n_split;

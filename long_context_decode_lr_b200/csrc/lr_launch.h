@@ -13,7 +13,7 @@ struct PackArgs;
 
 // General CUDA-core decode path (any supported shape, fp32 or bf16 storage).
 size_t decode_general_smem_bytes(int hd, int H, int G);
-size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split, int elem_bytes);
+size_t decode_combine_smem_bytes(int hd, int H, int G, int n_split, int elem_bytes, int n_tail);
 cudaError_t launch_decode_general(const DecodeArgs& a, lr_dtype dt, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecodeArgs& a, lr_dtype dt, cudaStream_t st);
 

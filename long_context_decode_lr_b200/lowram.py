@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "liblowram.so")
 LR_OK, LR_ERR_INVALID_ARG, LR_ERR_UNSUPPORTED, LR_ERR_WORKSPACE, LR_ERR_CUDA, LR_ERR_DEVICE_CHECK = range(6)
 LR_F32, LR_BF16 = 0, 1
 LR_BLOCK_TOKENS = 64
+LR_MAX_TAIL = 4096
 LR_DEVERR_BLOCK_RANGE, LR_DEVERR_BLOCK_ORDER, LR_DEVERR_RES_RANGE, LR_DEVERR_RES_ORDER, LR_DEVERR_PTR = 1, 2, 4, 8, 16
 LR_DEVERR_TIMEOUT, LR_DEVERR_LAUNCH = 32, 64
 
@@ -65,6 +66,8 @@ def library() -> ctypes.CDLL:
                                     _P, _P, _Z, _P]),
             "lr_decode_attn_noalloc": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _I, _P, _I, ctypes.c_float,
                                             _P, _P]),
+            "lr_decode_attn_tail": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _I, _P, _I, _P, _P, _I,
+                                         ctypes.c_float, _P, _P, _Z, _P]),
             "lr_topk_workspace_bytes": (_Z, [_I, _I, _I]),
             "lr_topk_tokens": (_I, [_P, _I, _I, _I, _P, _P, _Z, _P]),
             "lr_residual_block_ptr": (_I, [_P, _I, _I, _I, _P, _P]),
@@ -153,6 +156,17 @@ def lr_decode_attn_noalloc(shape, layer, n_q_heads, q, A, Bt, predictor: Predict
         ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
         _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, float(scale),
         _ptr(o), _stream(stream)))
+
+
+def lr_decode_attn_tail(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_idx, res_val,
+                        res_blk_ptr, k, block_list, n_sel, tail_K, tail_V, n_tail, scale, o, ws,
+                        stream=None) -> None:
+    """lr_decode_attn plus an exact recent-token tail tail_K / tail_V [B, Hkv, n_tail, hd]."""
+    _check(library().lr_decode_attn_tail(
+        ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
+        _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, _ptr(tail_K),
+        _ptr(tail_V), n_tail, float(scale), _ptr(o), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def lr_topk_workspace_bytes(n_segments: int, T: int, k: int) -> int:

@@ -130,7 +130,7 @@ def _rng(seed: int, *stream: int) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, *stream])))
 
 
-_STREAM_MODEL, _STREAM_SEQ, _STREAM_MLP, _STREAM_QUERY, _STREAM_BLOCKS, _STREAM_CACHE = range(6)
+_STREAM_MODEL, _STREAM_SEQ, _STREAM_MLP, _STREAM_QUERY, _STREAM_BLOCKS, _STREAM_CACHE, _STREAM_TAIL = range(7)
 _CHUNK = 4096  # tokens drawn per RNG call; fixed so that draws do not depend on memory limits
 
 
@@ -267,6 +267,21 @@ def queries(w: Workload, mw: ModelWeights, layer: int, batch: Optional[int] = No
         x = z @ mw.M + np.float32(0.05) * g.standard_normal((1, w.d_model), dtype=np.float32)
         q[b] = (x @ mw.W_Q[layer]).reshape(w.n_q_heads, w.head_dim)
     return q
+
+
+def tail_tokens(w: Workload, mw: ModelWeights, layer: int, n_tail: int, batch: Optional[int] = None):
+    """Keys and values [B, Hkv, n_tail, hd] of n_tail tokens generated after the cache was
+    packed: fresh hidden states of the workload's process through W_K, W_V of the layer."""
+    B = w.batch if batch is None else batch
+    K = np.empty((B, w.n_kv_heads, n_tail, w.head_dim), dtype=np.float32)
+    V = np.empty_like(K)
+    for b in range(B):
+        g = _rng(w.seed, _STREAM_TAIL, b, layer)
+        z = g.standard_normal((n_tail, w.dz), dtype=np.float32)
+        x = z @ mw.M + np.float32(0.05) * g.standard_normal((n_tail, w.d_model), dtype=np.float32)
+        K[b] = (x @ mw.W_K[layer]).reshape(n_tail, w.n_kv_heads, w.head_dim).transpose(1, 0, 2)
+        V[b] = (x @ mw.W_V[layer]).reshape(n_tail, w.n_kv_heads, w.head_dim).transpose(1, 0, 2)
+    return K, V
 
 
 def block_lists(w: Workload, batch: Optional[int] = None, n_sel: Optional[int] = None) -> np.ndarray:

@@ -139,7 +139,7 @@ def gpu_predictor(p: Problem) -> lr.Predictor:
     return lr.Predictor(s["W_lin"], s["W1"], s["b1"], s["W2"], s["b2"] if p.has_b2 else None, True)
 
 
-def gpu_decode(p: Problem, layer: int, q_st, use_ptr=True, scale=0.0, blocks=None, n_sel=None):
+def gpu_decode(p: Problem, layer: int, q_st, use_ptr=True, scale=0.0, blocks=None, n_sel=None, tail=None):
     w = p.w
     shape = shape_of(w)
     blocks = p.blocks if blocks is None else blocks
@@ -152,14 +152,20 @@ def gpu_decode(p: Problem, layer: int, q_st, use_ptr=True, scale=0.0, blocks=Non
     ws = lr.workspace(lr.lr_decode_workspace_bytes(shape, w.n_q_heads, n_sel))
     o = torch.empty((w.batch, w.n_q_heads, w.head_dim), dtype=TORCH_DT[w.dtype], device="cuda")
     pred = gpu_predictor(p)
-    lr.lr_decode_attn(shape, layer, w.n_q_heads, q_st, p.st["A"], p.st["Bt"], pred,
-                      p.st["idx"] if p.k else None, p.st["val"] if p.k else None,
-                      p.st["ptr"] if (use_ptr and p.k) else None, p.k, bl, n_sel, scale, o, ws)
+    if tail is None:
+        lr.lr_decode_attn(shape, layer, w.n_q_heads, q_st, p.st["A"], p.st["Bt"], pred,
+                          p.st["idx"] if p.k else None, p.st["val"] if p.k else None,
+                          p.st["ptr"] if (use_ptr and p.k) else None, p.k, bl, n_sel, scale, o, ws)
+    else:  # tail = (K, V) device tensors [B, Hkv, n_tail, hd] in the cache dtype
+        lr.lr_decode_attn_tail(shape, layer, w.n_q_heads, q_st, p.st["A"], p.st["Bt"], pred,
+                               p.st["idx"] if p.k else None, p.st["val"] if p.k else None,
+                               p.st["ptr"] if (use_ptr and p.k) else None, p.k, bl, n_sel,
+                               tail[0], tail[1], tail[0].shape[2], scale, o, ws)
     code = lr.lr_get_device_error(ws)
     return o.to(torch.float64).cpu().numpy(), code
 
 
-def oracle_decode(p: Problem, layer: int, q_ref, scale=0.0, blocks=None, heads=None):
+def oracle_decode(p: Problem, layer: int, q_ref, scale=0.0, blocks=None, heads=None, tail=None):
     w = p.w
     blocks = p.blocks if blocks is None else blocks
     sc = orc.default_scale(w.head_dim, scale)
@@ -169,7 +175,8 @@ def oracle_decode(p: Problem, layer: int, q_ref, scale=0.0, blocks=None, heads=N
         out[b] = orc.decode_sequence(q_ref[b], r["A"][b], r["Bt"][b], r["W_lin"][b], r["W1"][b], r["b1"][b],
                                      r["W2"][b], r["b2"][b] if p.has_b2 else None, layer, r["idx"][b],
                                      r["val"][b], None if blocks is None else blocks[b], sc,
-                                     w.n_kv_heads, w.head_dim)
+                                     w.n_kv_heads, w.head_dim,
+                                     None if tail is None else tail[0][b], None if tail is None else tail[1][b])
     return out
 
 

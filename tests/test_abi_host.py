@@ -113,3 +113,24 @@ def test_workspace_sizes_grow_with_work(lib):
     assert 0 < lib.lr_pack_workspace_bytes(ctypes.byref(s1), 10) < lib.lr_pack_workspace_bytes(ctypes.byref(s2), 10)
     assert lib.lr_decode_workspace_bytes(ctypes.byref(s1), 8, 0) >= 256
     assert lib.lr_decode_workspace_bytes(ctypes.byref(_shape(head_dim=12)), 8, 0) == 0
+
+
+def _decode_tail(lib, tail_K=FAKE, tail_V=FAKE, n_tail=16, ws_bytes=1 << 40):
+    shape, pred = _shape(), _pred()
+    return lib.lr_decode_attn_tail(ctypes.byref(shape), 0, 8, FAKE, FAKE, FAKE, ctypes.byref(pred), FAKE, FAKE,
+                                   None, 10, None, 0, tail_K, tail_V, n_tail, 0.0, FAKE, FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(n_tail=-1), lr.LR_ERR_INVALID_ARG),
+    (dict(n_tail=lr.LR_MAX_TAIL + 1), lr.LR_ERR_INVALID_ARG),
+    (dict(tail_K=None), lr.LR_ERR_INVALID_ARG),
+    (dict(tail_V=None), lr.LR_ERR_INVALID_ARG),
+    (dict(tail_V=FAKE + 8), lr.LR_ERR_INVALID_ARG),
+    (dict(ws_bytes=100), lr.LR_ERR_WORKSPACE),
+    (dict(tail_K=None, tail_V=None, n_tail=0, ws_bytes=100), lr.LR_ERR_WORKSPACE),  # no tail: NULL is fine
+])
+def test_decode_tail_rejects_bad_arguments(lib, kw, status):
+    """The tail arguments are checked on the host, before any launch."""
+    assert _decode_tail(lib, **kw) == status
+    assert lib.lr_last_error()
