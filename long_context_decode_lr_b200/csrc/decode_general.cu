@@ -228,15 +228,27 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
     const T* qp = (const T*)a.q + ((size_t)b * Hq + qh) * hd;
     for (int d = tid; d < hd; d += CT) qv[d] = to_f32(qp[d]);
     __syncthreads();
+    // one warp per tail token, lanes across the key's dims (coalesced rows), four tokens
+    // of a warp in flight at once
     const T* kt = (const T*)a.tail_K + ((size_t)b * a.Hkv + h) * nt * hd;
-    for (int t = tid; t < nt; t += CT) {
-      const T* kr = kt + (size_t)t * hd;
-      float s0 = 0.f, s1 = 0.f;
-      for (int d = 0; d < hd; d += 2) {
-        s0 = fmaf(qv[d], to_f32(kr[d]), s0);
-        s1 = fmaf(qv[d + 1], to_f32(kr[d + 1]), s1);
+    for (int t0 = warp; t0 < nt; t0 += 4 * (CT / 32)) {
+      float sv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * (CT / 32);
+        float acc_d = 0.f;
+        if (t < nt) {
+          const T* kr = kt + (size_t)t * hd;
+          for (int d = lane; d < hd; d += 32) acc_d = fmaf(qv[d], to_f32(kr[d]), acc_d);
+        }
+        sv[u] = acc_d;
       }
-      ts[t] = (s0 + s1) * a.scale;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u * (CT / 32);
+        const float v = warp_sum(sv[u]);
+        if (lane == 0 && t < nt) ts[t] = v * a.scale;
+      }
     }
   }
 
@@ -274,10 +286,19 @@ __global__ void __launch_bounds__(CT) decode_combine_kernel(DecodeArgs a) {
   __syncthreads();
   if (nt > 0) {  // tail values weighted by their softmax weights, this block's columns
     const T* vt = (const T*)a.tail_V + ((size_t)b * a.Hkv + h) * nt * hd + j0;
-    float av = 0.f;
-    if (lane < nj)
-      for (int t = warp; t < nt; t += CT / 32) av = fmaf(ts[t], to_f32(vt[(size_t)t * hd + lane]), av);
-    tred[warp * CJ + lane] = av;
+    float av[4] = {0.f, 0.f, 0.f, 0.f};
+    if (lane < nj) {
+      int t = warp;
+      for (; t + 3 * (CT / 32) < nt; t += 4 * (CT / 32)) {
+        float x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = to_f32(vt[(size_t)(t + u * (CT / 32)) * hd + lane]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) av[u] = fmaf(ts[t + u * (CT / 32)], x[u], av[u]);
+      }
+      for (; t < nt; t += CT / 32) av[0] = fmaf(ts[t], to_f32(vt[(size_t)t * hd + lane]), av[0]);
+    }
+    tred[warp * CJ + lane] = (av[0] + av[1]) + (av[2] + av[3]);
   }
   const int n_acc = hd + H + nj;
   for (int it = tid; it < L.n_ch * n_acc; it += CT) {
