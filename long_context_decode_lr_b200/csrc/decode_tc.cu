@@ -1,4 +1,6 @@
-// Tensor-core decode over the compressed cache (bf16 cache, head_dim 128, sm_100a).
+// Single-CTA tensor-core decode over the compressed cache (bf16 cache, head_dim 128,
+// sm_100a). The CTA-pair kernel (decode_pair.cu) is the default path for these shapes;
+// this one is the fallback (LOWRAM_DECODE_PATH=tensor), kept under the same parity tests.
 //
 // One CTA owns (split, KV-head pair, sequence) and walks 128-token tiles (two
 // 64-token blocks: consecutive blocks in full mode, entries of the pair's
@@ -17,7 +19,8 @@
 // The second-stage operands (k~, g, p and W1) are fp16: 11 significant bits keep the
 // rebuilt values within the attention tolerance even when one token dominates.
 // Roles: warp 0 issues TMA loads into a 3-stage ring (A, B_l and Qhat chunks of 64
-// rank columns, then W1 halves), warp 1 issues the MMAs, warps 2-5 run the epilogue.
+// rank columns, then W1 halves), warp 1 issues the MMAs, warps 2-9 run the epilogue
+// (two groups of four splitting the columns), warp 10 scatters the residual rows.
 // A prep kernel converts the layer's W1 to fp16, forms Qhat and (selective mode)
 // merges each pair's block lists. The split partials (m, l, sum p k~, sum p g,
 // sum p r) go to the same combine kernel as the general path. Every wait is bounded:
