@@ -239,6 +239,41 @@ def decode_sequence(q, A, Bt, W_lin, W1, b1, W2, b2, layer: int, res_idx, res_va
     return o
 
 
+def block_scores(q, A, Bt, layer: int, n_kv_heads: int, head_dim: int, scale: float,
+                 block: int = BLOCK) -> np.ndarray:
+    """Relevance of every 64-token block to the current query, per KV head: [Hkv, nblk].
+
+    The pages rebuild only the chunks the current query selects (explainer, paragraph on
+    prefill and decode costs; arXiv abstract) but their trained selector is not available.
+    Here a block's key is the mean of its reconstructed keys (the last block clipped at
+    T), and its score for KV head h is the largest scaled dot product with that mean over
+    the query heads h*G .. h*G+G-1 that read head h.
+    """
+    q = np.asarray(q, np.float64)
+    A = np.asarray(A, np.float64)
+    T = A.shape[0]
+    G = q.shape[0] // n_kv_heads
+    nblk = (T + block - 1) // block
+    out = np.empty((n_kv_heads, nblk), np.float64)
+    for h in range(n_kv_heads):
+        kt = reconstruct_keys(A, key_slice(Bt, layer, h, n_kv_heads, head_dim))
+        for j in range(nblk):
+            kbar = kt[j * block:min(T, (j + 1) * block)].mean(axis=0)
+            out[h, j] = max(float(q[h * G + g] @ kbar) * scale for g in range(G))
+    return out
+
+
+def select_blocks(scores, n_sel: int) -> np.ndarray:
+    """The n_sel blocks of highest score per KV head, ties to the lower block id, returned
+    in ascending order: [Hkv, n_sel] (the block-list layout lr_decode_attn reads)."""
+    scores = np.asarray(scores, np.float64)
+    out = np.empty((scores.shape[0], n_sel), np.int64)
+    for h in range(scores.shape[0]):
+        order = np.lexsort((np.arange(scores.shape[1]), -scores[h]))
+        out[h] = np.sort(order[:n_sel])
+    return out
+
+
 def default_scale(head_dim: int, scale: float) -> float:
     """The softmax scale: the given one when positive, else 1/sqrt(head_dim)."""
     return scale if scale > 0 else 1.0 / math.sqrt(head_dim)

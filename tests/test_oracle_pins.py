@@ -333,3 +333,42 @@ def test_tail_alone_and_tail_order():
     b = orc.decode_sequence(q, *args, None, 0.25, Hkv, hd, tK[:, perm], tV[:, perm])
     np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
     assert not np.allclose(a, orc.decode_sequence(q, *args, None, 0.25, Hkv, hd))
+
+
+def test_block_scores_are_rank_space_means_and_selection_is_brute_force():
+    """Block scores: the mean of a block's reconstructed keys equals the rank-space mean of
+    its A rows times the basis (linearity), so the score can be formed from block means
+    of A; a block whose keys are aligned with a query head wins; the selection is the
+    brute-force top-n_sel with ties to the lower block id, ascending."""
+    rng = np.random.default_rng(12)
+    L, Hkv, G, hd, T, r = 1, 2, 2, 16, 300, 24
+    K_group, V, pred = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])[:, :r]
+    A = orc.project_keys(K_group, Bt)
+    q = rng.standard_normal((Hkv * G, hd))
+    sc = orc.block_scores(q, A, Bt, 0, Hkv, hd, 0.5)
+    assert sc.shape == (Hkv, 5)
+    for h in range(Hkv):
+        Bh = orc.key_slice(Bt, 0, h, Hkv, hd)
+        for j in range(5):
+            abar = A[j * 64:min(T, j * 64 + 64)].mean(axis=0)   # the last block has 44 rows
+            want = max(0.5 * float(q[h * G + g] @ (Bh @ abar)) for g in range(G))
+            assert abs(sc[h, j] - want) <= 1e-12 * max(1.0, abs(want))
+    # a planted block: keys of block 3 of head 1 point along query head 3 (G = 2: head 1 reads 2, 3)
+    A2 = A.copy()
+    B1 = orc.key_slice(Bt, 0, 1, Hkv, hd)
+    A2[192:256] += 50.0 * (np.linalg.pinv(B1) @ q[3])
+    assert np.argmax(orc.block_scores(q, A2, Bt, 0, Hkv, hd, 1.0)[1]) == 3
+    # selection against brute force over all subsets, with ties
+    import itertools
+    s = np.array([[1.0, 3.0, 3.0, -2.0, 3.0, 0.5], [0.0, 0.0, 0.0, 0.0, 0.0, 0.0]])
+    for n_sel in range(0, 7):
+        got = orc.select_blocks(s, n_sel)
+        for h in range(2):
+            best = None
+            for sub in itertools.combinations(range(6), n_sel):
+                key = (sorted((-s[h, i] for i in sub)), list(sub))
+                if best is None or key < best[0]:
+                    best = (key, sub)
+            # the chosen set has the largest multiset of scores and, among equals, the lowest ids
+            assert list(got[h]) == sorted(best[1])
