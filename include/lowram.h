@@ -199,6 +199,33 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* shape, int32_t layer, int32_
                               const void* tail_V, int32_t n_tail, float scale, void* o,
                               void* ws, size_t ws_bytes, lr_stream_t stream);
 
+/* ------------------------------------------------------------------ block selection */
+
+/* Workspace bytes lr_select_blocks needs. */
+size_t lr_select_workspace_bytes(const lr_cache_shape* shape, int32_t n_q_heads);
+
+/*
+ * lr_select_blocks -- choose the 64-token blocks a decode step rebuilds (selective
+ * reconstruction: arXiv abstract; explainer, paragraph on prefill and decode costs, where
+ * only the chunks the current query selects are rebuilt). The pages' trained selector is
+ * not available; this one scores a block by its mean reconstructed key:
+ *   score[b, h, j] = max over the query heads hq = h G .. h G + G - 1 of
+ *                    scale * q[b, hq] . mean_{t in block j} k~_t,   k~_t = A[b, t] . B_l^h,
+ * the last block clipped at T, and returns per (b, h) the n_sel blocks of highest score,
+ * ties to the lower block id, in ascending order: the block_list layout of lr_decode_attn.
+ *
+ * Inputs:  q [B, Hq, hd]; A [B, T, r]; Bt [B, D, r]; 0 <= layer < L_g; n_q_heads a multiple of
+ *          Hkv with at most 8 query heads per KV head; 0 <= n_sel <= nblk; scale <= 0 selects
+ *          1/sqrt(hd); rank r <= 16384.
+ * Output:  block_list [B, Hkv, n_sel] int32 (not touched when n_sel == 0).
+ * Errors:  argument and shape errors on the host before any launch; LR_ERR_CUDA on a launch
+ *          failure. Scores are fp32: blocks whose scores differ by less than fp32 rounding may
+ *          be ordered either way.
+ */
+lr_status lr_select_blocks(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads, const void* q,
+                           const void* A, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
+                           void* ws, size_t ws_bytes, lr_stream_t stream);
+
 /* ------------------------------------------------------------------ single steps */
 
 /* Workspace bytes lr_topk_tokens needs. */

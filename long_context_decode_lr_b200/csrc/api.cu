@@ -206,6 +206,49 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* s, int32_t layer, int32_t n_
                      tail_K, tail_V, n_tail, scale, o, ws, ws_bytes, stream);
 }
 
+// ------------------------------------------------------------------ block selection
+
+size_t lr_select_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads) {
+  if (check_shape(s) != LR_OK || n_q_heads < 1) return 0;
+  const size_t nblk = (size_t)lr::ceil_div(s->T, LR_BLOCK_TOKENS);
+  const size_t qhat = (size_t)s->batch * n_q_heads * s->rank * sizeof(float);
+  const size_t scores = (size_t)s->batch * s->n_kv_heads * nblk * sizeof(float);
+  return 256 + ((qhat + 255) & ~(size_t)255) + ((scores + 255) & ~(size_t)255);
+}
+
+lr_status lr_select_blocks(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
+                           const void* A, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
+                           void* ws, size_t ws_bytes, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (layer < 0 || layer >= s->n_layers) return fail(LR_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, s->n_layers);
+  if (n_q_heads < 1 || n_q_heads % s->n_kv_heads) return fail(LR_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
+  if (n_q_heads / s->n_kv_heads > 8) return fail(LR_ERR_UNSUPPORTED, "more than 8 query heads per KV head");
+  if (s->rank > 16384) return fail(LR_ERR_UNSUPPORTED, "block selection supports rank <= 16384");
+  const int nblk = lr::ceil_div(s->T, LR_BLOCK_TOKENS);
+  if (n_sel < 0 || n_sel > nblk) return fail(LR_ERR_INVALID_ARG, "n_sel=%d outside [0, nblk=%d]", n_sel, nblk);
+  CHECK_PTR(q, "q");
+  CHECK_PTR(Bt, "Bt");
+  if (n_sel > 0) {
+    CHECK_PTR(A, "A");
+    CHECK_PTR(block_list, "block_list");
+  }
+  if ((st = check_ws(ws, ws_bytes, lr_select_workspace_bytes(s, n_q_heads))) != LR_OK) return st;
+  if (n_sel == 0 || s->batch == 0) return LR_OK;
+  lr::SelectArgs a{};
+  a.B = s->batch; a.T = s->T; a.L = s->n_layers; a.Hkv = s->n_kv_heads; a.G = n_q_heads / s->n_kv_heads;
+  a.hd = s->head_dim; a.r = s->rank; a.layer = layer; a.nblk = nblk; a.n_sel = n_sel;
+  a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)s->head_dim);
+  a.q = q; a.A = A; a.Bt = Bt;
+  const size_t qhat = (size_t)s->batch * n_q_heads * s->rank * sizeof(float);
+  a.qhat = (float*)((char*)ws + 256);
+  a.scores = (float*)((char*)ws + 256 + ((qhat + 255) & ~(size_t)255));
+  a.blocks_out = block_list;
+  const cudaError_t e = lr::launch_select_blocks(a, s->dtype, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block selection launch");
+  return LR_OK;
+}
+
 // ------------------------------------------------------------------ pack
 
 size_t lr_pack_workspace_bytes(const lr_cache_shape* s, int32_t k) {

@@ -87,6 +87,19 @@ __device__ __forceinline__ HeadPredictor<T> head_predictor(const DecodeArgs& a, 
   return p;
 }
 
+// Block selection (select.cu): scores of every 64-token block per (sequence, KV head) and
+// the top-n_sel block list.
+struct SelectArgs {
+  int B, T, L, Hkv, G, hd, r, layer, nblk, n_sel;
+  float scale;
+  const void* q;   // [B, Hq, hd]
+  const void* A;   // [B, T, r]
+  const void* Bt;  // [B, D, r]
+  float* qhat;     // workspace [B, Hkv, G, r]: scale * B_l^h q per query head
+  float* scores;   // workspace [B, Hkv, nblk]
+  int* blocks_out; // [B, Hkv, n_sel]
+};
+
 struct PackArgs {
   int B, T, L, Hkv, hd, r, H, D, k, nblk;
   int pred_per_seq;

@@ -10,6 +10,7 @@ namespace lr {
 
 struct DecodeArgs;
 struct PackArgs;
+struct SelectArgs;
 
 // General CUDA-core decode path (any supported shape, fp32 or bf16 storage).
 size_t decode_general_smem_bytes(int hd, int H, int G);
@@ -25,5 +26,8 @@ cudaError_t launch_pack_gather(const PackArgs& a, lr_dtype dt, cudaStream_t st);
 // Top-k token selection (radix select) and residual block pointers.
 cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st);
 cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_out, cudaStream_t st);
+
+// Block selection: mean-key block scores and their top-n_sel per (sequence, KV head).
+cudaError_t launch_select_blocks(const SelectArgs& a, lr_dtype dt, cudaStream_t st);
 
 }  // namespace lr

@@ -134,3 +134,31 @@ def test_decode_tail_rejects_bad_arguments(lib, kw, status):
     """The tail arguments are checked on the host, before any launch."""
     assert _decode_tail(lib, **kw) == status
     assert lib.lr_last_error()
+
+
+def _select(lib, shape=None, layer=0, hq=8, n_sel=4, ws=FAKE, ws_bytes=1 << 40, blocks=FAKE):
+    shape = _shape() if shape is None else shape
+    return lib.lr_select_blocks(ctypes.byref(shape), layer, hq, FAKE, FAKE, FAKE, n_sel, 0.0, blocks, ws,
+                                ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(layer=2), lr.LR_ERR_INVALID_ARG),
+    (dict(hq=7), lr.LR_ERR_INVALID_ARG),
+    (dict(hq=2 * 16), lr.LR_ERR_UNSUPPORTED),
+    (dict(n_sel=-1), lr.LR_ERR_INVALID_ARG),
+    (dict(n_sel=17), lr.LR_ERR_INVALID_ARG),          # T = 1000 has 16 blocks
+    (dict(blocks=None), lr.LR_ERR_INVALID_ARG),
+    (dict(ws=None), lr.LR_ERR_INVALID_ARG),
+    (dict(ws_bytes=100), lr.LR_ERR_WORKSPACE),
+    (dict(shape=_shape(rank=16392)), lr.LR_ERR_UNSUPPORTED),
+])
+def test_select_blocks_rejects_bad_arguments(lib, kw, status):
+    assert _select(lib, **kw) == status
+    assert lib.lr_last_error()
+
+
+def test_select_workspace_counts_queries_and_blocks(lib):
+    small, big = _shape(T=1000), _shape(T=64000)
+    assert lib.lr_select_workspace_bytes(ctypes.byref(small), 8) < lib.lr_select_workspace_bytes(ctypes.byref(big), 8)
+    assert lib.lr_select_workspace_bytes(ctypes.byref(small), 8) >= 256 + 8 * 128 * 4 + 2 * 16 * 4
