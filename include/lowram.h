@@ -29,7 +29,9 @@
  *     LR_ERR_CUDA means a launch failed (cudaGetLastError). Device-side data
  *     checks (out-of-range or unsorted indices) skip the offending entry and set
  *     bits in an error word inside the workspace; read it with
- *     lr_get_device_error. No kernel traps, asserts or spins.
+ *     lr_get_device_error. No kernel traps or asserts, and every wait inside a
+ *     kernel is bounded (on expiry the call's output is invalid and the error
+ *     word gets LR_DEVERR_TIMEOUT).
  *   - The last failing host-side check's message is available, per thread, from
  *     lr_last_error().
  *
@@ -89,7 +91,8 @@ typedef struct lr_cache_shape {
  * Value predictor f_theta of every (layer, KV head) of the group ("Predicting
  * the value cache from keys", paragraphs 2-3):
  *     v_hat = k W_lin^T + GELU(k W1^T + b1) W2^T + b2,   GELU(x) = x Phi(x) (erf form),
- * where k is the reconstructed key of one token and one KV head. Weights are in
+ * where k is the reconstructed key of one token and one KV head (the tensor-core decode
+ * kernels evaluate GELU in a tanh form within 2.7e-4 of the erf form). Weights are in
  * nn.Linear layout (out x in). With per_sequence = 1 every array has a leading
  * batch dimension [B, ...]; with 0 one predictor serves all sequences.
  *     W_lin [(B,) L_g, Hkv, hd, hd]     W1 [(B,) L_g, Hkv, H, hd]     b1 [(B,) L_g, Hkv, H]
