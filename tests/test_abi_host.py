@@ -162,3 +162,22 @@ def test_select_workspace_counts_queries_and_blocks(lib):
     small, big = _shape(T=1000), _shape(T=64000)
     assert lib.lr_select_workspace_bytes(ctypes.byref(small), 8) < lib.lr_select_workspace_bytes(ctypes.byref(big), 8)
     assert lib.lr_select_workspace_bytes(ctypes.byref(small), 8) >= 256 + 8 * 128 * 4 + 2 * 16 * 4
+
+
+def test_decode_path_override_changes_the_plan(lib, monkeypatch):
+    """bf16 / head_dim 128 caches plan the CTA-pair kernel; LOWRAM_DECODE_PATH forces the
+    single-CTA tensor-core or the CUDA-core plan instead (each has its own workspace layout)."""
+    shape = _shape(T=32768, n_layers=4, n_kv_heads=8, rank=1024)
+    sizes = {}
+    for path in ("pair", "tensor", "general"):
+        monkeypatch.setenv("LOWRAM_DECODE_PATH", path)
+        sizes[path] = lib.lr_decode_workspace_bytes(ctypes.byref(shape), 32, 0)
+    monkeypatch.delenv("LOWRAM_DECODE_PATH")
+    default = lib.lr_decode_workspace_bytes(ctypes.byref(shape), 32, 0)
+    assert default == sizes["pair"]
+    assert len(set(sizes.values())) == 3 and min(sizes.values()) > 0
+    f32 = _shape(T=32768, n_layers=4, n_kv_heads=8, rank=1024, dtype=lr.LR_F32)
+    monkeypatch.setenv("LOWRAM_DECODE_PATH", "pair")  # not available for fp32: the general plan
+    a = lib.lr_decode_workspace_bytes(ctypes.byref(f32), 32, 0)
+    monkeypatch.setenv("LOWRAM_DECODE_PATH", "general")
+    assert a == lib.lr_decode_workspace_bytes(ctypes.byref(f32), 32, 0)
