@@ -21,7 +21,12 @@ fp32 values held in float64). Sources, by page and section:
   by reconstruction error, one predictor per head; the "Where the memory
   actually goes" paragraph: the per-head storage budget.
 * arXiv 2611.07025 abstract page: only a selected subset of the cached pairs
-  is rebuilt at each decoding step (selective reconstruction).
+  is rebuilt at each decoding step (selective reconstruction); the predictor is
+  fitted at test time.
+* explainer, paragraph on prefill cost: the predictor is fitted to each context
+  with gradient steps (150 steps, a full fit of 300, 2 from a meta-learned start).
+* explainer, comparison table: LowRAM combined with quantisation keeps its
+  residuals at 2 bits per number.
 
 Readings where the pages are silent (each also listed in the design notes):
 the predictor sees the reconstructed key; a residual is the difference
@@ -34,7 +39,10 @@ with round-to-nearest-even.
 Parity pins: every function here is checked by ``tests/test_oracle_pins.py``
 against facts the pages or mathematics fix (Slim-Attention exactness, 100 %
 residual budget, full-rank keys, brute-force top-k, tabulated normal CDF
-values, a hand-computed predictor, the worked memory example).
+values, a hand-computed predictor, the worked memory example, column sums and
+the rank-space identity for block means, hand-computed 2-bit codes and the
+nearest-level property, finite-difference gradients and the least-squares limit
+of the fitting steps).
 """
 from __future__ import annotations
 
@@ -274,6 +282,22 @@ def select_blocks(scores, n_sel: int) -> np.ndarray:
     return out
 
 
+def block_means(A, block: int = BLOCK) -> np.ndarray:
+    """Mean of the A rows of every 64-token block, the last block clipped at T: [nblk, r].
+
+    The rebuilt key is linear in A, so the mean rebuilt key of block j for KV head h is
+    block_means(A)[j] . B_l^h (the block key that block_scores ranks): the block means
+    are query-independent and can be formed once, when the cache is packed.
+    """
+    A = np.asarray(A, np.float64)
+    T = A.shape[0]
+    nblk = (T + block - 1) // block
+    out = np.zeros((nblk, A.shape[1]), np.float64)
+    for j in range(nblk):
+        out[j] = A[j * block:min(T, (j + 1) * block)].mean(axis=0)
+    return out
+
+
 def default_scale(head_dim: int, scale: float) -> float:
     """The softmax scale: the given one when positive, else 1/sqrt(head_dim)."""
     return scale if scale > 0 else 1.0 / math.sqrt(head_dim)
@@ -307,3 +331,114 @@ def residual_budget(T: int, head_dim: int, ratio: float, hidden: int) -> float:
 def dense_cache_bytes_per_token(n_layers: int, n_kv_heads: int, head_dim: int, elem_bytes: int) -> int:
     """Bytes one token adds to an uncompressed K+V cache."""
     return n_layers * n_kv_heads * head_dim * 2 * elem_bytes
+
+
+# --------------------------------------------------------------------------- 2-bit residual rows
+
+def quantize_residual_rows(rows):
+    """2-bit codes of residual rows (explainer, comparison table: LowRAM + quantisation
+    stores its residuals with 2 bits per number). The pages name no quantiser; the reading
+    taken is the plain uniform one per row: four levels lo + c * step, c in {0, 1, 2, 3},
+    from the row's minimum lo to its maximum hi, step = (hi - lo) / 3, and each entry gets
+    the nearest level (ties to the even code). The code of an entry is an integer decided
+    in floating point, so it is taken in fp32, the precision of the kernel that packs the
+    rows: hi - lo, the step, x - lo and the quotient are each one correctly rounded fp32
+    operation; a row with step 0 (all entries equal) gets code 0 everywhere.
+
+    rows [n, hd] (exact values of the storage type) -> codes [n, hd] uint8, lo [n] fp32,
+    step [n] fp32.
+    """
+    x = np.asarray(rows, np.float64).astype(np.float32)
+    n = x.shape[0]
+    codes = np.zeros(x.shape, np.uint8)
+    lo = np.zeros(n, np.float32)
+    step = np.zeros(n, np.float32)
+    for i in range(n):
+        row = x[i]
+        if row.size == 0:
+            continue
+        l, h = np.float32(row.min()), np.float32(row.max())
+        st = np.float32(np.float32(h - l) / np.float32(3.0))
+        lo[i], step[i] = l, st
+        if st > 0:
+            t = (row - l).astype(np.float32) / st
+            codes[i] = np.clip(np.rint(t.astype(np.float32)), 0, 3).astype(np.uint8)
+    return codes, lo, step
+
+
+def dequantize_residual_rows(codes, lo, step) -> np.ndarray:
+    """The residual rows a decode step adds: lo + code * step per entry, [n, hd] fp64."""
+    return (np.asarray(lo, np.float64)[:, None]
+            + np.asarray(codes, np.float64) * np.asarray(step, np.float64)[:, None])
+
+
+def pack_2bit(codes) -> np.ndarray:
+    """Byte layout of the codes: entry 4i + s of a row sits in bits 2s..2s+1 of byte i."""
+    c = np.asarray(codes, np.uint8)
+    n, hd = c.shape
+    c4 = c.reshape(n, hd // 4, 4).astype(np.uint32)
+    return (c4[..., 0] | (c4[..., 1] << 2) | (c4[..., 2] << 4) | (c4[..., 3] << 6)).astype(np.uint8)
+
+
+def unpack_2bit(packed, hd: int) -> np.ndarray:
+    """Inverse of pack_2bit: [n, hd / 4] bytes -> [n, hd] codes."""
+    p = np.asarray(packed, np.uint8).astype(np.uint32)
+    out = np.stack([(p >> (2 * s)) & 3 for s in range(4)], axis=-1)
+    return out.reshape(p.shape[0], hd).astype(np.uint8)
+
+
+# --------------------------------------------------------------------------- test-time fitting
+
+def gelu_grad(x) -> np.ndarray:
+    """Derivative of the erf-form GELU: Phi(x) + x phi(x)."""
+    x = np.asarray(x, np.float64)
+    Phi = 0.5 * (1.0 + erf(x / math.sqrt(2.0)))
+    phi = np.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+    return Phi + x * phi
+
+
+def predictor_loss(kt, v, params) -> float:
+    """Mean squared value error of the predictor over the context's tokens and the head's
+    entries: mean_{t, j} (v_hat_t[j] - v_t[j])^2. The explainer (paragraph 2 and the
+    paragraph on prefill cost) fits the per-head network to this context with gradient
+    steps; it does not name the loss, and the mean squared error is the plainest reading
+    (the same per-token error that ranks the residuals, averaged)."""
+    vh = predict_values(kt, params["W_lin"], params["W1"], params["b1"], params["W2"], params.get("b2"))
+    d = vh - np.asarray(v, np.float64)
+    return float(np.mean(d * d))
+
+
+def predictor_grads(kt, v, params):
+    """Gradients of predictor_loss with respect to every predictor parameter (W_lin, W1,
+    b1, W2 and b2 when the predictor has one), by the chain rule through
+    v_hat = k W_lin^T + GELU(k W1^T + b1) W2^T + b2."""
+    kt = np.asarray(kt, np.float64)
+    v = np.asarray(v, np.float64)
+    W_lin, W1, b1, W2 = (np.asarray(params[n], np.float64) for n in ("W_lin", "W1", "b1", "W2"))
+    b2 = params.get("b2")
+    u = kt @ W1.T + b1
+    g = gelu(u)
+    vh = kt @ W_lin.T + g @ W2.T
+    if b2 is not None:
+        vh = vh + np.asarray(b2, np.float64)
+    dv = 2.0 * (vh - v) / v.size          # d loss / d v_hat
+    du = (dv @ W2) * gelu_grad(u)         # d loss / d u
+    out = {"W_lin": dv.T @ kt, "W1": du.T @ kt, "b1": du.sum(axis=0), "W2": dv.T @ g}
+    if b2 is not None:
+        out["b2"] = dv.sum(axis=0)
+    return out
+
+
+def fit_predictor(kt, v, params, n_steps: int, lr: float):
+    """Test-time fitting of one head's predictor to the context's own (reconstructed key,
+    value) pairs: n_steps of full-batch gradient descent on predictor_loss from the given
+    start (the pseudoinverse initialisation, or a previous fit). Explainer, paragraph on
+    prefill cost: 150 gradient steps per context, a full fit of 300, two steps from a
+    meta-learned start; the pages name neither the optimiser nor the step size, so the
+    plainest reading is taken: theta <- theta - lr * grad, with lr given by the caller."""
+    p = {n: (None if a is None else np.array(a, np.float64, copy=True)) for n, a in params.items()}
+    for _ in range(n_steps):
+        gr = predictor_grads(kt, v, p)
+        for n, d in gr.items():
+            p[n] = p[n] - lr * d
+    return p

@@ -3,7 +3,10 @@ of the oracle (never in the oracle itself), runs the pin tests against that copy
 subprocess and expects them to fail: a dropped bias, a flipped residual sign, a transposed
 weight, the wrong tie rule, the wrong head slice or GQA map, a missing scale, a dropped
 residual, the tanh GELU, an ignored exact tail, a block score that sums instead of averaging,
-a block selection that breaks ties upwards.
+a block selection that breaks ties upwards, block means over an unclipped last block, a
+quantiser that floors or uses four steps or the wrong bit order, a GELU derivative without
+its x phi term, a flipped or mis-scaled gradient, a W1 gradient from the wrong rows, an
+untrained b2, a fitting step that climbs.
 """
 import os
 import shutil
@@ -37,6 +40,21 @@ MUTATIONS = {
                          "kbar = kt[j * block:min(T, (j + 1) * block)].sum(axis=0) / block"),
     "block ties upwards": ("order = np.lexsort((np.arange(scores.shape[1]), -scores[h]))",
                            "order = np.lexsort((-np.arange(scores.shape[1]), -scores[h]))"),
+    "block means over a full block": ("out[j] = A[j * block:min(T, (j + 1) * block)].mean(axis=0)",
+                                      "out[j] = A[j * block:min(T, (j + 1) * block)].sum(axis=0) / block"),
+    "quantiser floors": ("codes[i] = np.clip(np.rint(t.astype(np.float32)), 0, 3).astype(np.uint8)",
+                         "codes[i] = np.clip(np.floor(t.astype(np.float32)), 0, 3).astype(np.uint8)"),
+    "quantiser four steps": ("st = np.float32(np.float32(h - l) / np.float32(3.0))",
+                             "st = np.float32(np.float32(h - l) / np.float32(4.0))"),
+    "code bit order": ("return (c4[..., 0] | (c4[..., 1] << 2) | (c4[..., 2] << 4) | (c4[..., 3] << 6)).astype(np.uint8)",
+                       "return (c4[..., 3] | (c4[..., 2] << 2) | (c4[..., 1] << 4) | (c4[..., 0] << 6)).astype(np.uint8)"),
+    "GELU derivative without x phi": ("    return Phi + x * phi", "    return Phi"),
+    "gradient sign": ("dv = 2.0 * (vh - v) / v.size", "dv = 2.0 * (v - vh) / v.size"),
+    "loss averaged over tokens only": ("dv = 2.0 * (vh - v) / v.size", "dv = 2.0 * (vh - v) / v.shape[0]"),
+    "W1 gradient from the wrong side": ('out = {"W_lin": dv.T @ kt, "W1": du.T @ kt,',
+                                        'out = {"W_lin": dv.T @ kt, "W1": (du.T @ kt) * 0.0 + du.T @ kt[::-1],'),
+    "b2 not trained": ('        out["b2"] = dv.sum(axis=0)', '        out["b2"] = 0.0 * dv.sum(axis=0)'),
+    "fit step ascends": ("            p[n] = p[n] - lr * d", "            p[n] = p[n] + lr * d"),
 }
 
 

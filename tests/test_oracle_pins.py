@@ -372,3 +372,145 @@ def test_block_scores_are_rank_space_means_and_selection_is_brute_force():
                     best = (key, sub)
             # the chosen set has the largest multiset of scores and, among equals, the lowest ids
             assert list(got[h]) == sorted(best[1])
+
+
+# ----------------------------------------------------------------------------- block means
+
+def test_block_means_against_column_sums_and_block_scores():
+    """Block means: a constant block gives that constant; the last block is clipped at T;
+    summing mean x block size over the blocks gives the column sums of A; and scoring a
+    block through its mean A row equals the oracle's block score over reconstructed keys
+    (the rebuild is linear)."""
+    rng = np.random.default_rng(21)
+    T, r = 300, 10
+    A = rng.standard_normal((T, r))
+    A[64:128] = np.arange(r)                       # block 1 is constant
+    m = orc.block_means(A)
+    assert m.shape == (5, r)
+    np.testing.assert_array_equal(m[1], np.arange(r, dtype=np.float64))
+    sizes = np.array([64, 64, 64, 64, 44.0])
+    np.testing.assert_allclose((m * sizes[:, None]).sum(axis=0), A.sum(axis=0), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(m[4] * 44.0, A[256:].sum(axis=0), rtol=1e-12, atol=1e-12)
+    L, Hkv, G, hd = 1, 2, 3, 8
+    K_group, _, _ = _group_problem(rng, L=L, Hkv=Hkv, G=G, hd=hd, T=T)
+    Bt = _orthogonal(rng, K_group.shape[1])[:, :12]
+    A2 = orc.project_keys(K_group, Bt)
+    q = rng.standard_normal((Hkv * G, hd))
+    sc = orc.block_scores(q, A2, Bt, 0, Hkv, hd, 0.3)
+    mb = orc.block_means(A2)
+    for h in range(Hkv):
+        Bh = orc.key_slice(Bt, 0, h, Hkv, hd)
+        want = np.max(0.3 * (q[h * G:(h + 1) * G] @ Bh) @ mb.T, axis=0)
+        np.testing.assert_allclose(sc[h], want, rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- 2-bit residual rows
+
+def test_quantize_residual_rows_hand_values():
+    rows = np.array([
+        [0.0, 1.0, 2.0, 3.0, 3.0, 2.0, 1.0, 0.0],      # lo 0, step 1: the codes are the values
+        [0.0, 0.5, 1.5, 2.5, 3.0, 3.0, 3.0, 3.0],      # ties: 0.5 -> 0, 1.5 -> 2, 2.5 -> 2 (even)
+        [2.0, 2.0, 2.0, 2.0, 2.0, 2.0, 2.0, 2.0],      # constant row: step 0, codes 0
+        [-3.0, 0.0, 3.0, 1.5, -3.0, -3.0, -3.0, -3.0],  # lo -3, step 2: 1.5, 3, 2.25 -> 2, 3, 2
+    ])
+    codes, lo, step = orc.quantize_residual_rows(rows)
+    np.testing.assert_array_equal(codes[0], [0, 1, 2, 3, 3, 2, 1, 0])
+    np.testing.assert_array_equal(codes[1], [0, 0, 2, 2, 3, 3, 3, 3])
+    np.testing.assert_array_equal(codes[2], np.zeros(8))
+    np.testing.assert_array_equal(codes[3], [0, 2, 3, 2, 0, 0, 0, 0])
+    np.testing.assert_array_equal(lo, [0.0, 0.0, 2.0, -3.0])
+    np.testing.assert_array_equal(step, [1.0, 1.0, 0.0, 2.0])
+    back = orc.dequantize_residual_rows(codes, lo, step)
+    np.testing.assert_array_equal(back[0], rows[0])
+    np.testing.assert_array_equal(back[2], rows[2])
+    assert back[3, 1] == 1.0 and back[3, 2] == 3.0
+
+
+def test_quantize_residual_rows_nearest_level_and_bound():
+    """Every entry gets a nearest level (within fp32 rounding of a tie), the row minimum and
+    maximum get codes 0 and 3, and the round trip is within half a step."""
+    rng = np.random.default_rng(5)
+    rows = orc.round_bf16(rng.standard_normal((200, 128)) * np.exp(rng.uniform(-4, 4, (200, 1))))
+    codes, lo, step = orc.quantize_residual_rows(rows)
+    back = orc.dequantize_residual_rows(codes, lo, step)
+    for i in range(rows.shape[0]):
+        levels = lo[i] + np.arange(4) * np.float64(step[i])
+        dist = np.abs(rows[i][:, None] - levels[None, :])
+        got = dist[np.arange(128), codes[i]]
+        assert np.all(got <= dist.min(axis=1) + 1e-6 * step[i])
+        assert codes[i][np.argmin(rows[i])] == 0 and codes[i][np.argmax(rows[i])] == 3
+        assert np.max(np.abs(back[i] - rows[i])) <= 0.5 * step[i] * (1 + 1e-5) + 1e-6 * np.abs(rows[i]).max()
+
+
+def test_pack_2bit_layout():
+    codes = np.array([[1, 2, 3, 0, 3, 3, 3, 3]], np.uint8)
+    packed = orc.pack_2bit(codes)
+    assert packed.tolist() == [[1 + (2 << 2) + (3 << 4), 255]]
+    rng = np.random.default_rng(3)
+    c = rng.integers(0, 4, (9, 128)).astype(np.uint8)
+    np.testing.assert_array_equal(orc.unpack_2bit(orc.pack_2bit(c), 128), c)
+
+
+# ----------------------------------------------------------------------------- test-time fitting
+
+def _fit_problem(rng, T=13, hd=3, H=4, b2=True):
+    kt = rng.standard_normal((T, hd))
+    v = rng.standard_normal((T, hd))
+    p = {"W_lin": rng.standard_normal((hd, hd)), "W1": rng.standard_normal((H, hd)),
+         "b1": rng.standard_normal(H), "W2": rng.standard_normal((hd, H)),
+         "b2": rng.standard_normal(hd) if b2 else None}
+    return kt, v, p
+
+
+@pytest.mark.parametrize("b2", [True, False])
+def test_predictor_grads_match_finite_differences(b2):
+    rng = np.random.default_rng(31)
+    kt, v, p = _fit_problem(rng, b2=b2)
+    gr = orc.predictor_grads(kt, v, p)
+    assert set(gr) == {n for n, a in p.items() if a is not None}
+    eps = 1e-6
+    for name, g in gr.items():
+        num = np.zeros_like(g)
+        for ix in np.ndindex(g.shape):
+            pp = {n: (None if a is None else a.copy()) for n, a in p.items()}
+            pm = {n: (None if a is None else a.copy()) for n, a in p.items()}
+            pp[name][ix] += eps
+            pm[name][ix] -= eps
+            num[ix] = (orc.predictor_loss(kt, v, pp) - orc.predictor_loss(kt, v, pm)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-9, err_msg=name)
+
+
+def test_fit_zero_steps_descent_and_exact_start():
+    rng = np.random.default_rng(32)
+    kt, v, p = _fit_problem(rng, T=40, hd=4, H=5)
+    same = orc.fit_predictor(kt, v, p, 0, 0.1)
+    for n in p:
+        np.testing.assert_array_equal(same[n], p[n])
+    l0 = orc.predictor_loss(kt, v, p)
+    assert orc.predictor_loss(kt, v, orc.fit_predictor(kt, v, p, 1, 1e-3)) < l0
+    assert orc.predictor_loss(kt, v, orc.fit_predictor(kt, v, p, 20, 1e-2)) < orc.predictor_loss(
+        kt, v, orc.fit_predictor(kt, v, p, 1, 1e-2))
+    # a start that already predicts every value exactly is a stationary point
+    p0 = dict(p, W2=np.zeros_like(p["W2"]))
+    v0 = kt @ p0["W_lin"].T + p0["b2"]
+    fitted = orc.fit_predictor(kt, v0, p0, 5, 0.5)
+    for n in p0:
+        np.testing.assert_array_equal(fitted[n], p0[n])
+
+
+def test_fit_linear_branch_converges_to_least_squares():
+    """With the nonlinear branch switched off (W1 = 0, b1 = 0, W2 = 0 give zero gradients
+    to W1, b1 and W2), gradient descent fits the linear map and b2 by least squares."""
+    rng = np.random.default_rng(33)
+    T, hd, H = 40, 3, 2
+    kt = rng.standard_normal((T, hd))
+    v = rng.standard_normal((T, hd))
+    p = {"W_lin": np.zeros((hd, hd)), "W1": np.zeros((H, hd)), "b1": np.zeros(H),
+         "W2": np.zeros((hd, H)), "b2": np.zeros(hd)}
+    fitted = orc.fit_predictor(kt, v, p, 3000, 1.0)
+    X = np.concatenate([kt, np.ones((T, 1))], axis=1)
+    sol, *_ = np.linalg.lstsq(X, v, rcond=None)
+    np.testing.assert_allclose(fitted["W_lin"], sol[:hd].T, atol=1e-8)
+    np.testing.assert_allclose(fitted["b2"], sol[hd], atol=1e-8)
+    np.testing.assert_array_equal(fitted["W1"], 0.0)
+    np.testing.assert_array_equal(fitted["W2"], 0.0)
