@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define LR_ABI_VERSION 1
+#define LR_ABI_VERSION 2
 #define LR_BLOCK_TOKENS 64
 
 typedef void* lr_stream_t; /* cudaStream_t */
@@ -204,6 +204,18 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* shape, int32_t layer, int32_
 
 /* ------------------------------------------------------------------ block selection */
 
+/*
+ * lr_block_means -- the mean A row of every 64-token block of the packed cache:
+ *   Abar[b, j] = mean_{t in block j} A[b, t],   the last block clipped at T.
+ * The rebuilt key is linear in A, so Abar[b, j] . B_l^h is the mean rebuilt key of block j
+ * for every layer and KV head of the group. Abar does not depend on the query: compute it
+ * once after lr_pack_prefill and pass it to every lr_select_blocks call on that cache.
+ * Inputs: A [B, T, r] (cache dtype). Output: Abar [B, nblk, r] fp32 (1/64 of A's rows).
+ * Errors: shape errors and NULL / misaligned pointers on the host; LR_ERR_CUDA on a launch
+ * failure. Needs no workspace.
+ */
+lr_status lr_block_means(const lr_cache_shape* shape, const void* A, float* Abar, lr_stream_t stream);
+
 /* Workspace bytes lr_select_blocks needs. */
 size_t lr_select_workspace_bytes(const lr_cache_shape* shape, int32_t n_q_heads);
 
@@ -213,21 +225,23 @@ size_t lr_select_workspace_bytes(const lr_cache_shape* shape, int32_t n_q_heads)
  * only the chunks the current query selects are rebuilt). The pages' trained selector is
  * not available; this one scores a block by its mean reconstructed key:
  *   score[b, h, j] = max over the query heads hq = h G .. h G + G - 1 of
- *                    scale * q[b, hq] . mean_{t in block j} k~_t,   k~_t = A[b, t] . B_l^h,
- * the last block clipped at T, and returns per (b, h) the n_sel blocks of highest score,
- * ties to the lower block id, in ascending order: the block_list layout of lr_decode_attn.
+ *                    scale * q[b, hq] . mean_{t in block j} k~_t
+ *                  = max_hq (scale * B_l^h q[b, hq]) . Abar[b, j],   k~_t = A[b, t] . B_l^h,
+ * and returns per (b, h) the n_sel blocks of highest score, ties to the lower block id, in
+ * ascending order: the block_list layout of lr_decode_attn. The list is exactly the top
+ * n_sel of the returned fp32 scores.
  *
- * Inputs:  q [B, Hq, hd]; A [B, T, r]; Bt [B, D, r]; 0 <= layer < L_g; n_q_heads a multiple of
- *          Hkv with at most 8 query heads per KV head; 0 <= n_sel <= nblk; scale <= 0 selects
- *          1/sqrt(hd); rank r <= 16384.
- * Output:  block_list [B, Hkv, n_sel] int32 (not touched when n_sel == 0).
+ * Inputs:  q [B, Hq, hd]; Abar [B, nblk, r] fp32 from lr_block_means; Bt [B, D, r];
+ *          0 <= layer < L_g; n_q_heads a multiple of Hkv with at most 8 query heads per KV
+ *          head; 0 <= n_sel <= nblk; scale <= 0 selects 1/sqrt(hd).
+ * Outputs: block_list [B, Hkv, n_sel] int32 (not touched when n_sel == 0);
+ *          scores_out [B, Hkv, nblk] fp32 or NULL (the scores the list was taken from).
  * Errors:  argument and shape errors on the host before any launch; LR_ERR_CUDA on a launch
- *          failure. Scores are fp32: blocks whose scores differ by less than fp32 rounding may
- *          be ordered either way.
+ *          failure. Scores are fp32 (a rank-space dot product accumulated in fp32).
  */
 lr_status lr_select_blocks(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads, const void* q,
-                           const void* A, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
-                           void* ws, size_t ws_bytes, lr_stream_t stream);
+                           const float* Abar, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
+                           float* scores_out, void* ws, size_t ws_bytes, lr_stream_t stream);
 
 /* ------------------------------------------------------------------ single steps */
 
@@ -274,9 +288,10 @@ lr_status lr_residual_block_ptr(const int32_t* idx, int32_t n_segments, int32_t 
  *   - All calls on a device share the array and each call clears the part that must start
  *     at zero; calls that overlap on the GPU (different streams, or host threads without
  *     ordering) race on it.
- *   - Device-side data checks write the shared array's error word, which this entry point
- *     does not expose; use lr_decode_attn with a workspace when you need
- *     lr_get_device_error.
+ *   - Device-side data checks write the shared array's error word; lr_get_device_error
+ *     with ws = NULL reads it (the word of the last call on the current device).
+ *   - The array's address is looked up once per device and kept for the life of the
+ *     process: do not use this entry point on a device after cudaDeviceReset there.
  * Argument meaning, layouts, ownership and the other error behaviour: as lr_decode_attn.
  */
 lr_status lr_decode_attn_noalloc(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
@@ -291,7 +306,8 @@ lr_status lr_decode_attn_noalloc(const lr_cache_shape* shape, int32_t layer, int
 /* Copies the device error word of the last call that used `ws` into *code and
  * synchronises `stream`. Returns LR_OK when the word is 0, LR_ERR_DEVICE_CHECK when it
  * is not, LR_ERR_CUDA when the copy fails. Every call that takes a workspace clears
- * the word when it starts. */
+ * the word when it starts. ws = NULL reads the word of the last lr_decode_attn_noalloc
+ * call on the current device. */
 lr_status lr_get_device_error(const void* ws, lr_stream_t stream, int32_t* code);
 
 const char* lr_status_string(lr_status status);

@@ -84,6 +84,7 @@ int current_sm_count() {
 namespace lr {
 // Records a message for lr_last_error() (used by entry points defined in other files).
 void set_last_error(const char* msg) { snprintf(g_msg, sizeof(g_msg), "%s", msg); }
+lr_status noalloc_scratch_address(void** out);
 }  // namespace lr
 
 extern "C" {
@@ -105,7 +106,12 @@ const char* lr_status_string(lr_status s) {
 }
 
 lr_status lr_get_device_error(const void* ws, lr_stream_t stream, int32_t* code) {
-  if (!ws || !code) return fail(LR_ERR_INVALID_ARG, "ws and code must not be NULL");
+  if (!code) return fail(LR_ERR_INVALID_ARG, "code must not be NULL");
+  if (!ws) {  // the scratch array of lr_decode_attn_noalloc on the current device
+    void* p = nullptr;
+    if (lr::noalloc_scratch_address(&p) != LR_OK) return fail(LR_ERR_CUDA, "locating the allocation-free scratch");
+    ws = p;
+  }
   int32_t v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -216,33 +222,43 @@ size_t lr_select_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads) {
   return 256 + ((qhat + 255) & ~(size_t)255) + ((scores + 255) & ~(size_t)255);
 }
 
+lr_status lr_block_means(const lr_cache_shape* s, const void* A, float* Abar, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (s->batch == 0 || s->T == 0) return LR_OK;
+  CHECK_PTR(A, "A");
+  CHECK_PTR(Abar, "Abar");
+  const cudaError_t e = lr::launch_block_means(A, s->batch, s->T, s->rank, s->dtype, Abar, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "block means launch");
+  return LR_OK;
+}
+
 lr_status lr_select_blocks(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
-                           const void* A, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
-                           void* ws, size_t ws_bytes, lr_stream_t stream) {
+                           const float* Abar, const void* Bt, int32_t n_sel, float scale, int32_t* block_list,
+                           float* scores_out, void* ws, size_t ws_bytes, lr_stream_t stream) {
   lr_status st = check_shape(s);
   if (st != LR_OK) return st;
   if (layer < 0 || layer >= s->n_layers) return fail(LR_ERR_INVALID_ARG, "layer %d outside [0, %d)", layer, s->n_layers);
   if (n_q_heads < 1 || n_q_heads % s->n_kv_heads) return fail(LR_ERR_INVALID_ARG, "n_q_heads must be a positive multiple of n_kv_heads");
   if (n_q_heads / s->n_kv_heads > 8) return fail(LR_ERR_UNSUPPORTED, "more than 8 query heads per KV head");
-  if (s->rank > 16384) return fail(LR_ERR_UNSUPPORTED, "block selection supports rank <= 16384");
   const int nblk = lr::ceil_div(s->T, LR_BLOCK_TOKENS);
   if (n_sel < 0 || n_sel > nblk) return fail(LR_ERR_INVALID_ARG, "n_sel=%d outside [0, nblk=%d]", n_sel, nblk);
   CHECK_PTR(q, "q");
   CHECK_PTR(Bt, "Bt");
-  if (n_sel > 0) {
-    CHECK_PTR(A, "A");
-    CHECK_PTR(block_list, "block_list");
-  }
+  CHECK_OPT_PTR(scores_out, "scores_out");
+  const bool work = (n_sel > 0 || scores_out) && nblk > 0;
+  if (work) CHECK_PTR(Abar, "Abar");
+  if (n_sel > 0) CHECK_PTR(block_list, "block_list");
   if ((st = check_ws(ws, ws_bytes, lr_select_workspace_bytes(s, n_q_heads))) != LR_OK) return st;
-  if (n_sel == 0 || s->batch == 0) return LR_OK;
+  if (!work || s->batch == 0) return LR_OK;
   lr::SelectArgs a{};
   a.B = s->batch; a.T = s->T; a.L = s->n_layers; a.Hkv = s->n_kv_heads; a.G = n_q_heads / s->n_kv_heads;
   a.hd = s->head_dim; a.r = s->rank; a.layer = layer; a.nblk = nblk; a.n_sel = n_sel;
   a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)s->head_dim);
-  a.q = q; a.A = A; a.Bt = Bt;
+  a.q = q; a.abar = Abar; a.Bt = Bt;
   const size_t qhat = (size_t)s->batch * n_q_heads * s->rank * sizeof(float);
   a.qhat = (float*)((char*)ws + 256);
-  a.scores = (float*)((char*)ws + 256 + ((qhat + 255) & ~(size_t)255));
+  a.scores = scores_out ? scores_out : (float*)((char*)ws + 256 + ((qhat + 255) & ~(size_t)255));
   a.blocks_out = block_list;
   const cudaError_t e = lr::launch_select_blocks(a, s->dtype, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "block selection launch");

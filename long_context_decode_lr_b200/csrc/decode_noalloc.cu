@@ -10,8 +10,11 @@
 // The array lives on every GPU that loads the library until the process exits, and all
 // calls on a device share it. The first call on a device looks up the array's device
 // address with cudaGetSymbolAddress (host code cannot use the array's name as a device
-// pointer); make that first call before any stream capture. Calls that overlap on the
-// GPU (different streams, or host threads without ordering) race on the array.
+// pointer); make that first call before any stream capture. The address is kept for the
+// life of the process, so the entry point must not be used on a device after
+// cudaDeviceReset there. Calls that overlap on the GPU (different streams, or host threads
+// without ordering) race on the array. lr_get_device_error with a NULL workspace reads the
+// array's error word (that of the last call on the current device).
 #include <atomic>
 
 #include <cuda_runtime.h>
@@ -34,7 +37,11 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
 std::atomic<void*> g_scratch_addr[kMaxDevices];
 
-lr_status scratch_address(void** out) {
+}  // namespace
+
+namespace lr {
+// Device address of the current device's scratch array (looked up once per device).
+lr_status noalloc_scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LR_ERR_CUDA;
   void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
@@ -45,8 +52,7 @@ lr_status scratch_address(void** out) {
   *out = p;
   return LR_OK;
 }
-
-}  // namespace
+}  // namespace lr
 
 extern "C" lr_status lr_decode_attn_noalloc(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
                                             const void* q, const void* A, const void* Bt,
@@ -62,7 +68,7 @@ extern "C" lr_status lr_decode_attn_noalloc(const lr_cache_shape* shape, int32_t
     return LR_ERR_WORKSPACE;
   }
   void* ws = nullptr;
-  const lr_status st = scratch_address(&ws);
+  const lr_status st = lr::noalloc_scratch_address(&ws);
   if (st != LR_OK) return st;
   return lr_decode_attn(shape, layer, n_q_heads, q, A, Bt, predictor, res_idx, res_val, res_blk_ptr, k, block_list,
                         n_sel, scale, o, ws, kScratchBytes, stream);

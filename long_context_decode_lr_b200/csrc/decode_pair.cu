@@ -81,7 +81,8 @@ enum Bar {
 };
 static_assert(N_BARS * 8 <= 320, "barrier area");
 
-constexpr float kGeluC1 = 0.80015708f;  // tanh-form GELU, minimax fit (csrc/gelu_fit.py)
+constexpr float kGeluC1 = 0.80015708f;  // tanh-form GELU: c1, c3 minimise the largest error
+                                        // against x Phi(x) on [-10, 10] (2.71e-4)
 constexpr float kGeluC3 = 0.03470089f;
 
 __device__ __forceinline__ float gelu_f32(float x) {

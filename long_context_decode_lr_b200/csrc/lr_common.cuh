@@ -92,12 +92,12 @@ __device__ __forceinline__ HeadPredictor<T> head_predictor(const DecodeArgs& a, 
 struct SelectArgs {
   int B, T, L, Hkv, G, hd, r, layer, nblk, n_sel;
   float scale;
-  const void* q;   // [B, Hq, hd]
-  const void* A;   // [B, T, r]
-  const void* Bt;  // [B, D, r]
-  float* qhat;     // workspace [B, Hkv, G, r]: scale * B_l^h q per query head
-  float* scores;   // workspace [B, Hkv, nblk]
-  int* blocks_out; // [B, Hkv, n_sel]
+  const void* q;       // [B, Hq, hd]
+  const float* abar;   // [B, nblk, r] block means of A
+  const void* Bt;      // [B, D, r]
+  float* qhat;         // workspace [B, Hkv, G, r]: scale * B_l^h q per query head
+  float* scores;       // [B, Hkv, nblk]: the caller's scores_out, or workspace
+  int* blocks_out;     // [B, Hkv, n_sel]
 };
 
 struct PackArgs {

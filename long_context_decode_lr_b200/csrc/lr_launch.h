@@ -27,7 +27,9 @@ cudaError_t launch_pack_gather(const PackArgs& a, lr_dtype dt, cudaStream_t st);
 cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st);
 cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_out, cudaStream_t st);
 
-// Block selection: mean-key block scores and their top-n_sel per (sequence, KV head).
+// Block selection: block means of A (once per packed cache), mean-key block scores and
+// their top-n_sel per (sequence, KV head).
+cudaError_t launch_block_means(const void* A, int B, int T, int r, lr_dtype dt, float* abar, cudaStream_t st);
 cudaError_t launch_select_blocks(const SelectArgs& a, lr_dtype dt, cudaStream_t st);
 
 }  // namespace lr

@@ -11,7 +11,7 @@ namespace lr {
 struct DecodeArgs;
 struct PackArgs;
 
-enum class DecodePath { General = 0, Tensor = 1, Pair = 2 };
+enum class DecodePath { General = 0, Pair = 2 };
 
 struct DecodePlan {
   DecodePath path;
@@ -19,9 +19,9 @@ struct DecodePlan {
   int n_pairs;       // pair path: CTA pairs per (sequence, KV head)
   int part_stride;   // floats per split partial
   size_t part_off;   // byte offset of the partials in the workspace
-  size_t sched_off;  // byte offset of the tensor path's block schedule
-  size_t w1h_off;    // byte offset of the tensor path's fp16 copy of the layer's W1
-  size_t qhat_off;   // byte offset of the tensor path's Qhat operand
+  size_t sched_off;  // byte offset of the pair path's block schedule
+  size_t w1h_off;    // byte offset of the pair path's fp16 copy of the layer's W1
+  size_t qhat_off;   // byte offset of the pair path's Qhat operand
   size_t ws_bytes;   // total workspace
 };
 
@@ -32,7 +32,6 @@ struct PackPlan {
   size_t ws_bytes;
 };
 
-bool decode_tc_supported(const lr_cache_shape& s, int n_q_heads);
 bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads);
 DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);
 PackPlan plan_pack(const lr_cache_shape& s, int k);

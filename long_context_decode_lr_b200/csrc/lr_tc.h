@@ -10,34 +10,6 @@
 namespace lr {
 namespace tc {
 
-struct TcArgs {
-  int B, T, L, Hkv, G, H, r;
-  int layer, k, nblk, pred_per_seq;
-  int n_hp;          // KV-head pairs
-  int n_split;       // CTAs per (sequence, head pair)
-  float scale;
-  const __nv_bfloat16* q;        // [B, Hq, 128]
-  const __nv_bfloat16* b1;       // [(B,) L, Hkv, H]
-  const __nv_bfloat16* Bt;       // [B, D, r]
-  __nv_bfloat16* qhat;           // workspace: [B, n_hp, 4*MG, r] scale * B_l^h q as bf16 hi/lo rows
-  const __nv_bfloat16* W1;       // [(B,) L, Hkv, H, 128]
-  __half* W1h;                   // workspace: [(B,) Hkv, H, 128] fp16 copy of the layer's W1
-  int w1_seqs;                   // 1, or B when each sequence has its own predictor
-  const int* res_idx;            // [B, L, Hkv, k]
-  const __nv_bfloat16* res_val;  // [B, L, Hkv, k, 128]
-  const int* res_ptr;            // [B, L, Hkv, nblk + 1] or null
-  const int* sched;              // selective mode: [B, n_hp, sched_stride]; null in full mode
-  int sched_stride;              // 1 + 2 * n_sel
-  float* partials;               // [B, Hq, n_split, part_stride]
-  int part_stride;
-  int* err;
-};
-
-// Rows of the Qhat operand per (sequence, head pair): 2 heads x (hi, lo) x 4 or 8 query heads.
-int qhat_rows(int G);
-cudaError_t launch_decode_tc(const TcArgs& a, const CUtensorMap& mA, const CUtensorMap& mB, const CUtensorMap& mQ,
-                             const CUtensorMap& mW1, const int* blocks, int n_sel, cudaStream_t st);
-
 // Pair kernel (2-CTA clusters, one KV head per pair; see decode_pair.cu).
 struct PairArgs {
   int B, T, L, Hkv, G, H, r;

@@ -43,12 +43,6 @@ bool tile_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank
 }
 }  // namespace
 
-bool decode_tc_supported(const lr_cache_shape& s, int n_q_heads) {
-  const int G = n_q_heads / s.n_kv_heads;
-  return s.dtype == LR_BF16 && s.head_dim == 128 && (s.hidden == 128 || s.hidden == 256) && s.rank % 64 == 0 &&
-         s.n_kv_heads % 2 == 0 && G >= 1 && G <= 8 && s.T > 0;
-}
-
 bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads) {
   const int G = n_q_heads / s.n_kv_heads;
   return s.dtype == LR_BF16 && s.head_dim == 128 && (s.hidden == 128 || s.hidden == 256) && s.rank % 64 == 0 &&
@@ -56,16 +50,13 @@ bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads) {
 }
 
 namespace {
-// Kernel family for the decode call: the CTA-pair kernel where the shape allows it, then
-// the single-CTA tensor-core kernel, then the CUDA-core kernel. LOWRAM_DECODE_PATH
-// (= "pair", "tensor" or "general") restricts the choice for testing; a path the shape does
-// not support is never taken.
+// Kernel family for the decode call: the CTA-pair tensor-core kernel where the shape allows
+// it, else the CUDA-core kernel. LOWRAM_DECODE_PATH=general forces the CUDA-core kernel for
+// every shape (a supported option, documented in lowram.h); "pair" or unset keeps the default.
 DecodePath choose_path(const lr_cache_shape& s, int n_q_heads) {
   const char* env = getenv("LOWRAM_DECODE_PATH");
-  const bool want_pair = !env || !strcmp(env, "pair");
-  const bool want_tc = !env || !strcmp(env, "tensor") || !strcmp(env, "pair");
+  const bool want_pair = !env || strcmp(env, "general") != 0;
   if (want_pair && decode_pair_supported(s, n_q_heads)) return DecodePath::Pair;
-  if (want_tc && decode_tc_supported(s, n_q_heads)) return DecodePath::Tensor;
   return DecodePath::General;
 }
 }  // namespace
@@ -99,28 +90,6 @@ DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm
     p.ws_bytes = align256(p.qhat_off + qhat_bytes);
     return p;
   }
-  if (path == DecodePath::Tensor) {
-    p.path = DecodePath::Tensor;
-    const int n_hp = s.n_kv_heads / 2;
-    const int rows = s.batch * n_hp;
-    const int max_tiles = ceil_div(n_sel > 0 ? (2 * n_sel < nblk ? 2 * n_sel : nblk) : nblk, 2);
-    int n_split = rows > 0 ? (sm_count + rows / 2) / rows : 1;
-    if (n_split > max_tiles) n_split = max_tiles;
-    if (n_split < 1) n_split = 1;
-    p.n_split = n_split;
-    p.part_stride = 4 + 2 * s.head_dim + s.hidden;
-    p.part_off = 256;
-    const size_t part_bytes = (size_t)s.batch * n_q_heads * n_split * p.part_stride * sizeof(float);
-    p.sched_off = align256(p.part_off + part_bytes);
-    // the schedule region is always reserved: an empty selected-block list still writes a count
-    const size_t sched_bytes = (size_t)rows * (1 + 2 * (size_t)(n_sel > 0 ? n_sel : 0)) * sizeof(int);
-    p.w1h_off = align256(p.sched_off + sched_bytes);
-    const size_t w1h_bytes = (size_t)s.batch * s.n_kv_heads * s.hidden * s.head_dim * 2;
-    p.qhat_off = align256(p.w1h_off + w1h_bytes);
-    const size_t qhat_bytes = (size_t)rows * tc::qhat_rows(n_q_heads / s.n_kv_heads) * s.rank * 2;
-    p.ws_bytes = align256(p.qhat_off + qhat_bytes);
-    return p;
-  }
   p.path = DecodePath::General;
   const int units = n_sel > 0 ? n_sel : nblk;
   const int per_row = s.batch * s.n_kv_heads;
@@ -150,52 +119,6 @@ PackPlan plan_pack(const lr_cache_shape& s, int k) {
 
 cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype dt, cudaStream_t st) {
   cudaError_t e;
-  if (plan.path == DecodePath::Tensor) {
-    tc::TcArgs t{};
-    t.B = a.B; t.T = a.T; t.L = a.L; t.Hkv = a.Hkv; t.G = a.G; t.H = a.H; t.r = a.r;
-    t.layer = a.layer; t.k = a.k; t.nblk = a.nblk; t.pred_per_seq = a.pred_per_seq;
-    t.n_hp = a.Hkv / 2;
-    t.n_split = plan.n_split;
-    t.scale = a.scale;
-    t.q = (const __nv_bfloat16*)a.q;
-    t.b1 = (const __nv_bfloat16*)a.b1;
-    t.W1 = (const __nv_bfloat16*)a.W1;
-    t.Bt = (const __nv_bfloat16*)a.Bt;
-    t.qhat = (__nv_bfloat16*)((char*)a.err + plan.qhat_off);
-    t.W1h = (__half*)((char*)a.err + plan.w1h_off);
-    t.w1_seqs = a.pred_per_seq ? a.B : 1;
-    t.res_idx = a.res_idx;
-    t.res_val = (const __nv_bfloat16*)a.res_val;
-    t.res_ptr = a.res_ptr;
-    t.sched = a.blocks ? (const int*)((char*)a.err + plan.sched_off) : nullptr;
-    t.sched_stride = 1 + 2 * a.n_sel;
-    t.partials = a.partials;
-    t.part_stride = plan.part_stride;
-    t.err = a.err;
-    const cuuint64_t D = (cuuint64_t)a.L * a.Hkv * a.hd;
-    CUtensorMap mA, mB, mQ, mW1;
-    const cuuint64_t q_rows = (cuuint64_t)tc::qhat_rows(a.G);
-    const cuuint64_t dQ[2] = {(cuuint64_t)a.r, (cuuint64_t)a.B * t.n_hp * q_rows};
-    const cuuint64_t sQ[1] = {(cuuint64_t)a.r * 2};
-    const cuuint32_t bQ[2] = {64, (cuuint32_t)q_rows};
-    const cuuint64_t dA[3] = {(cuuint64_t)a.r, (cuuint64_t)a.T, (cuuint64_t)a.B};
-    const cuuint64_t sA[2] = {(cuuint64_t)a.r * 2, (cuuint64_t)a.T * a.r * 2};
-    const cuuint32_t bA[3] = {64, 64, 1};
-    const cuuint64_t dB[3] = {(cuuint64_t)a.r, D, (cuuint64_t)a.B};
-    const cuuint64_t sB[2] = {(cuuint64_t)a.r * 2, D * a.r * 2};
-    const cuuint32_t bB[3] = {64, 128, 1};
-    const cuuint64_t w1_rows = (cuuint64_t)t.w1_seqs * a.Hkv * a.H;
-    const cuuint64_t dW[2] = {(cuuint64_t)a.hd, w1_rows};
-    const cuuint64_t sW[1] = {(cuuint64_t)a.hd * 2};
-    const cuuint32_t bW[2] = {64, 128};
-    if (!tile_map(&mA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.A, 3, dA, sA, bA) ||
-        !tile_map(&mB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Bt, 3, dB, sB, bB) ||
-        !tile_map(&mQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, t.qhat, 2, dQ, sQ, bQ) ||
-        !tile_map(&mW1, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, t.W1h, 2, dW, sW, bW))
-      return cudaErrorInvalidValue;
-    if ((e = tc::launch_decode_tc(t, mA, mB, mQ, mW1, a.blocks, a.n_sel, st)) != cudaSuccess) return e;
-    return launch_decode_combine(a, dt, st);
-  }
   if (plan.path == DecodePath::Pair) {
     tc::PairArgs t{};
     t.B = a.B; t.T = a.T; t.L = a.L; t.Hkv = a.Hkv; t.G = a.G; t.H = a.H; t.r = a.r;

@@ -2,11 +2,12 @@
 // rebuilds (selective reconstruction, arXiv abstract; "Predicting the value cache from
 // keys", paragraph on prefill and decode costs). The pages' trained selector is not
 // available; a block's key is the mean of its rebuilt keys and its score for KV head h is
-//   s_j = max_g scale * q_g . mean_{t in block j} k~_t = max_g Qhat_g . mean_{t in block j} A_t,
-// with Qhat_g = scale * B_l^h q_g (the mean commutes with the linear key rebuild, so the
-// score needs one mean of A rows per block and one rank-space dot product per query head).
-// The n_sel blocks of highest score per (sequence, KV head) are then chosen by the exact
-// top-k of topk.cu (ties to the lower block id, ascending).
+//   s_j = max_g scale * q_g . mean_{t in block j} k~_t = max_g Qhat_g . Abar_j,
+// with Qhat_g = scale * B_l^h q_g and Abar_j the mean of the block's A rows (the mean
+// commutes with the linear key rebuild). Abar does not depend on the query: it is formed
+// once per packed cache (block_means_kernel), so a selection step reads 1/64 of A. The n_sel
+// blocks of highest score per (sequence, KV head) are then chosen by the exact top-k of
+// topk.cu (ties to the lower block id, ascending).
 #include "lr_common.cuh"
 #include "lr_launch.h"
 
@@ -15,85 +16,165 @@ namespace {
 
 constexpr int SEL_THREADS = 256;
 
-__device__ __forceinline__ float sel_warp_sum(float v) {
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+// 8 consecutive storage elements as fp32 (one 16-byte load for bf16, two for fp32).
+template <typename T>
+__device__ __forceinline__ void load8(const T* p, float (&v)[8]);
+template <>
+__device__ __forceinline__ void load8<__nv_bfloat16>(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+template <>
+__device__ __forceinline__ void load8<float>(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Qhat [B, Hkv, G, r] fp32: one block per (KV head, sequence), threads over rank columns.
+// Abar [B, nblk, r] fp32: one CTA per (block, sequence); a thread owns 8 rank columns and
+// sums the block's rows (up to 64) with four independent partial sums.
+template <typename T>
+__global__ void __launch_bounds__(SEL_THREADS) block_means_kernel(const T* __restrict__ A, int T_len, int r,
+                                                                  float* __restrict__ abar) {
+  const int j = blockIdx.x, b = blockIdx.y;
+  const int t0 = j * kBlock, n = min(T_len, t0 + kBlock) - t0;
+  const float inv_n = 1.f / (float)n;
+  const T* src = A + ((size_t)b * T_len + t0) * r;
+  float* dst = abar + ((size_t)b * gridDim.x + j) * r;
+  for (int c = threadIdx.x * 8; c < r; c += SEL_THREADS * 8) {
+    float s[4][8] = {};
+    int t = 0;
+    for (; t + 4 <= n; t += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        float v[8];
+        load8<T>(src + (size_t)(t + u) * r + c, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[u][i] += v[i];
+      }
+    }
+    for (; t < n; ++t) {
+      float v[8];
+      load8<T>(src + (size_t)t * r + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[0][i] += v[i];
+    }
+    float4 o0, o1;
+    o0.x = ((s[0][0] + s[1][0]) + (s[2][0] + s[3][0])) * inv_n;
+    o0.y = ((s[0][1] + s[1][1]) + (s[2][1] + s[3][1])) * inv_n;
+    o0.z = ((s[0][2] + s[1][2]) + (s[2][2] + s[3][2])) * inv_n;
+    o0.w = ((s[0][3] + s[1][3]) + (s[2][3] + s[3][3])) * inv_n;
+    o1.x = ((s[0][4] + s[1][4]) + (s[2][4] + s[3][4])) * inv_n;
+    o1.y = ((s[0][5] + s[1][5]) + (s[2][5] + s[3][5])) * inv_n;
+    o1.z = ((s[0][6] + s[1][6]) + (s[2][6] + s[3][6])) * inv_n;
+    o1.w = ((s[0][7] + s[1][7]) + (s[2][7] + s[3][7])) * inv_n;
+    reinterpret_cast<float4*>(dst + c)[0] = o0;
+    reinterpret_cast<float4*>(dst + c)[1] = o1;
+  }
+}
+
+// Qhat [B, Hkv * G, r] fp32: one CTA per (64 rank columns, KV head, sequence). Thread
+// (dg, c) sums every fourth key dim for rank column c; a 4-way reduction in shared memory.
 template <typename T>
 __global__ void __launch_bounds__(SEL_THREADS) select_qhat_kernel(SelectArgs a) {
-  extern __shared__ float qs[];  // [G][hd], scaled queries
-  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  __shared__ float qs[8][256];
+  __shared__ float part[4][64][9];
+  const int jc = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int G = a.G, hd = a.hd, r = a.r;
   const T* q = (const T*)a.q + ((size_t)b * a.Hkv + h) * G * hd;
-  for (int i = tid; i < G * hd; i += SEL_THREADS) qs[i] = to_f32(q[i]) * a.scale;
+  for (int i = tid; i < G * hd; i += SEL_THREADS) qs[i / hd][i % hd] = to_f32(q[i]) * a.scale;
   __syncthreads();
-  const size_t D = (size_t)a.L * a.Hkv * hd;
-  const T* bt = (const T*)a.Bt + (size_t)b * D * r + (size_t)(a.layer * a.Hkv + h) * hd * r;
-  float* out = a.qhat + ((size_t)b * a.Hkv + h) * G * r;
-  for (int j = tid; j < r; j += SEL_THREADS) {
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int d = 0; d < hd; ++d) {
-      const float v = to_f32(bt[(size_t)d * r + j]);
+  const int c = tid & 63, dg = tid >> 6;
+  const int j = jc * 64 + c;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (j < r) {
+    const size_t D = (size_t)a.L * a.Hkv * hd;
+    const T* bt = (const T*)a.Bt + (size_t)b * D * r + (size_t)(a.layer * a.Hkv + h) * hd * r + j;
+    for (int d = dg; d < hd; d += 4) {
+      const float v = to_f32(bt[(size_t)d * r]);
 #pragma unroll
       for (int g = 0; g < 8; ++g)
-        if (g < G) acc[g] = fmaf(v, qs[g * hd + d], acc[g]);
+        if (g < G) acc[g] = fmaf(v, qs[g][d], acc[g]);
     }
-#pragma unroll
-    for (int g = 0; g < 8; ++g)
-      if (g < G) out[(size_t)g * r + j] = acc[g];
   }
+#pragma unroll
+  for (int g = 0; g < 8; ++g) part[dg][c][g] = acc[g];
+  __syncthreads();
+  if (dg != 0 || j >= r) return;
+  float* out = a.qhat + ((size_t)b * a.Hkv + h) * G * r + j;
+#pragma unroll
+  for (int g = 0; g < 8; ++g)
+    if (g < G) out[(size_t)g * r] = (part[0][c][g] + part[1][c][g]) + (part[2][c][g] + part[3][c][g]);
 }
 
-// Scores [B, Hkv, nblk]: one CTA per (block, sequence). The block's mean A row goes to
-// shared memory; each warp then takes (KV head, query head) pairs, one rank-space dot
-// product each, and the maximum over a head's query heads is the block's score.
-template <typename T>
+constexpr int kScBlocks = 32;  // blocks per CTA (4 per warp)
+constexpr int kScPairs = 32;   // (KV head, query head) pairs per pass: one per lane
+constexpr int kScCols = 128;   // rank columns staged per pass
+static_assert(kScBlocks == kScPairs && kScBlocks == 4 * SEL_THREADS / 32, "staging loop and warp split");
+
+// Scores [B, Hkv, nblk]: one CTA per 32 blocks of a sequence. Lane l of every warp owns the
+// (KV head, query head) pair l of the current pass and accumulates its dot products with the
+// warp's 4 block means; rank columns are staged 128 at a time (Qhat rows padded against bank
+// conflicts, block means read as broadcasts).
 __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a) {
-  extern __shared__ float abar[];  // [r], then [Hkv * G] dot products
-  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int r = a.r, G = a.G, Hkv = a.Hkv;
-  const int t0 = j * kBlock, t1 = min(a.T, t0 + kBlock);
-  const T* A = (const T*)a.A + ((size_t)b * a.T + t0) * r;
-  const float inv_n = 1.f / (float)(t1 - t0);
-  for (int c = tid; c < r; c += SEL_THREADS) {
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    int t = 0;
-    for (; t + 4 <= t1 - t0; t += 4) {
+  __shared__ float qs[kScPairs][kScCols + 1];
+  __shared__ float as[kScBlocks][kScCols];
+  __shared__ float dots[kScBlocks][kScPairs + 1];
+  const int j0 = blockIdx.x * kScBlocks, b = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int r = a.r, G = a.G, P = a.Hkv * G;
+  const int nb = min(kScBlocks, a.nblk - j0);
+  const float* qh = a.qhat + (size_t)b * P * r;
+  const float* ab = a.abar + ((size_t)b * a.nblk + j0) * r;
+  const int pass = (kScPairs / G) * G;  // whole heads per pass: a head never straddles two
+  for (int p0 = 0; p0 < P; p0 += pass) {
+    const int np = min(pass, P - p0);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c0 = 0; c0 < r; c0 += kScCols) {
+      const int nc = min(kScCols, r - c0);
+      __syncthreads();
+      for (int i = tid; i < kScPairs * kScCols; i += SEL_THREADS) {
+        const int p = i / kScCols, c = i % kScCols;
+        qs[p][c] = (p < np && c < nc) ? qh[(size_t)(p0 + p) * r + c0 + c] : 0.f;
+        as[p][c] = (p < nb && c < nc) ? ab[(size_t)p * r + c0 + c] : 0.f;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int c = 0; c < kScCols; ++c) {
+        const float qv = qs[lane][c];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) s[u] += to_f32(A[(size_t)(t + u) * r + c]);
+        for (int i = 0; i < 4; ++i) acc[i] = fmaf(qv, as[warp * 4 + i][c], acc[i]);
+      }
     }
-    for (; t < t1 - t0; ++t) s[0] += to_f32(A[(size_t)t * r + c]);
-    abar[c] = ((s[0] + s[1]) + (s[2] + s[3])) * inv_n;
-  }
-  __syncthreads();
-  float* dots = abar + r;
-  for (int p = warp; p < Hkv * G; p += SEL_THREADS / 32) {
-    const float* qh = a.qhat + ((size_t)b * Hkv * G + p) * r;
-    float acc = 0.f;
-    for (int c = lane; c < r; c += 32) acc = fmaf(qh[c], abar[c], acc);
-    acc = sel_warp_sum(acc);
-    if (lane == 0) dots[p] = acc;
-  }
-  __syncthreads();
-  for (int h = tid; h < Hkv; h += SEL_THREADS) {
-    float m = dots[h * G];
-    for (int g = 1; g < G; ++g) m = fmaxf(m, dots[h * G + g]);
-    a.scores[((size_t)b * Hkv + h) * a.nblk + j] = m;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dots[warp * 4 + i][lane] = acc[i];
+    __syncthreads();
+    // per (block, head of this pass): the largest dot product over the head's query heads
+    const int nh = np / G;
+    for (int x = tid; x < kScBlocks * kScPairs; x += SEL_THREADS) {
+      const int blk = x / kScPairs, hl = x % kScPairs;
+      if (blk >= nb || hl >= nh) continue;
+      float m = dots[blk][hl * G];
+      for (int g = 1; g < G; ++g) m = fmaxf(m, dots[blk][hl * G + g]);
+      a.scores[((size_t)b * a.Hkv + p0 / G + hl) * a.nblk + j0 + blk] = m;
+    }
   }
 }
 
 template <typename T>
 cudaError_t launch_select_t(const SelectArgs& a, cudaStream_t st) {
-  const size_t qs_bytes = (size_t)a.G * a.hd * sizeof(float);
-  select_qhat_kernel<T><<<dim3(a.Hkv, a.B), SEL_THREADS, qs_bytes, st>>>(a);
+  select_qhat_kernel<T><<<dim3((a.r + 63) / 64, a.Hkv, a.B), SEL_THREADS, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t sc_bytes = ((size_t)a.r + (size_t)a.Hkv * a.G) * sizeof(float);
-  e = cudaFuncSetAttribute(select_score_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sc_bytes);
-  if (e != cudaSuccess) return e;
-  select_score_kernel<T><<<dim3(a.nblk, a.B), SEL_THREADS, sc_bytes, st>>>(a);
+  select_score_kernel<<<dim3((a.nblk + kScBlocks - 1) / kScBlocks, a.B), SEL_THREADS, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_topk(a.scores, a.B * a.Hkv, a.nblk, a.n_sel, a.blocks_out, st);
 }
@@ -103,6 +184,17 @@ cudaError_t launch_select_t(const SelectArgs& a, cudaStream_t st) {
 cudaError_t launch_select_blocks(const SelectArgs& a, lr_dtype dt, cudaStream_t st) {
   if (a.B == 0 || a.nblk == 0) return cudaSuccess;
   return dt == LR_BF16 ? launch_select_t<__nv_bfloat16>(a, st) : launch_select_t<float>(a, st);
+}
+
+cudaError_t launch_block_means(const void* A, int B, int T, int r, lr_dtype dt, float* abar, cudaStream_t st) {
+  const int nblk = ceil_div(T, kBlock);
+  if (B == 0 || nblk == 0) return cudaSuccess;
+  const dim3 grid(nblk, B);
+  if (dt == LR_BF16)
+    block_means_kernel<__nv_bfloat16><<<grid, SEL_THREADS, 0, st>>>((const __nv_bfloat16*)A, T, r, abar);
+  else
+    block_means_kernel<float><<<grid, SEL_THREADS, 0, st>>>((const float*)A, T, r, abar);
+  return cudaGetLastError();
 }
 
 }  // namespace lr

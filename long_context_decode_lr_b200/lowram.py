@@ -69,7 +69,8 @@ def library() -> ctypes.CDLL:
             "lr_decode_attn_tail": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _I, _P, _I, _P, _P, _I,
                                          ctypes.c_float, _P, _P, _Z, _P]),
             "lr_select_workspace_bytes": (_Z, [S, _I]),
-            "lr_select_blocks": (_I, [S, _I, _I, _P, _P, _P, _I, ctypes.c_float, _P, _P, _Z, _P]),
+            "lr_block_means": (_I, [S, _P, _P, _P]),
+            "lr_select_blocks": (_I, [S, _I, _I, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P, _Z, _P]),
             "lr_topk_workspace_bytes": (_Z, [_I, _I, _I]),
             "lr_topk_tokens": (_I, [_P, _I, _I, _I, _P, _P, _Z, _P]),
             "lr_residual_block_ptr": (_I, [_P, _I, _I, _I, _P, _P]),
@@ -175,11 +176,19 @@ def lr_select_workspace_bytes(shape: lr_cache_shape, n_q_heads: int) -> int:
     return library().lr_select_workspace_bytes(ctypes.byref(shape), n_q_heads)
 
 
-def lr_select_blocks(shape, layer, n_q_heads, q, A, Bt, n_sel, scale, block_list, ws, stream=None) -> None:
-    """The n_sel blocks per (sequence, KV head) whose mean rebuilt key best matches the query."""
+def lr_block_means(shape, A, Abar, stream=None) -> None:
+    """Abar [B, nblk, r] fp32: the mean A row of every 64-token block (query-independent)."""
+    _check(library().lr_block_means(ctypes.byref(shape), _ptr(A), _ptr(Abar), _stream(stream)))
+
+
+def lr_select_blocks(shape, layer, n_q_heads, q, Abar, Bt, n_sel, scale, block_list, ws, scores_out=None,
+                     stream=None) -> None:
+    """The n_sel blocks per (sequence, KV head) whose mean rebuilt key best matches the query;
+    scores_out [B, Hkv, nblk] fp32 (optional) receives the scores the list was taken from."""
     _check(library().lr_select_blocks(
-        ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), n_sel, float(scale), _ptr(block_list),
-        _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+        ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(Abar), _ptr(Bt), n_sel, float(scale),
+        _ptr(block_list), _ptr(scores_out), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def lr_topk_workspace_bytes(n_segments: int, T: int, k: int) -> int:

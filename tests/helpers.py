@@ -19,8 +19,11 @@ from oracle import lowram_oracle as orc
 
 TORCH_DT = {"bf16": torch.bfloat16, "f32": torch.float32}
 
-# Attention-output tolerance: relative L2 and max-abs error against the fp64 oracle
-# (bf16 storage, fp32 accumulation).
+# Attention-output tolerance against the fp64 oracle (bf16 storage, fp32 accumulation):
+# relative L2 <= 1e-2 and max-abs <= 2e-2 * max(1, max|ref|). The absolute bound is stated
+# for outputs of unit scale. Every floating result carries a relative error, and a bf16
+# output alone is rounded to 8 significant bits (at |o| >= 8 half a bf16 step already
+# exceeds 2e-2), so beyond |o| = 1 the max-abs bound grows with the output's magnitude.
 REL_L2 = 1e-2
 MAX_ABS = 2e-2
 
@@ -185,9 +188,10 @@ def assert_attention_close(got, ref, rel_l2=REL_L2, max_abs=MAX_ABS):
     nref = np.linalg.norm(ref)
     rel = np.linalg.norm(diff) / max(nref, 1e-30)
     mab = np.abs(diff).max() if diff.size else 0.0
+    bound = max_abs * max(1.0, float(np.abs(ref).max()) if ref.size else 1.0)
     assert np.all(np.isfinite(got)), "non-finite output"
-    print(f"[attention parity] rel_l2={rel:.3e} max_abs={mab:.3e}")
-    assert rel <= rel_l2 and mab <= max_abs, f"rel_l2={rel:.3e} max_abs={mab:.3e}"
+    print(f"[attention parity] rel_l2={rel:.3e} max_abs={mab:.3e} (bound {bound:.3e})")
+    assert rel <= rel_l2 and mab <= bound, f"rel_l2={rel:.3e} max_abs={mab:.3e} bound={bound:.3e}"
     return rel, mab
 
 

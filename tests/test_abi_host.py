@@ -36,7 +36,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.lr_abi_version() == 1
+    assert lib.lr_abi_version() == 2
     assert lib.lr_status_string(lr.LR_ERR_WORKSPACE) == b"workspace too small"
 
 
@@ -136,10 +136,11 @@ def test_decode_tail_rejects_bad_arguments(lib, kw, status):
     assert lib.lr_last_error()
 
 
-def _select(lib, shape=None, layer=0, hq=8, n_sel=4, ws=FAKE, ws_bytes=1 << 40, blocks=FAKE):
+def _select(lib, shape=None, layer=0, hq=8, n_sel=4, ws=FAKE, ws_bytes=1 << 40, blocks=FAKE, abar=FAKE,
+            scores=None):
     shape = _shape() if shape is None else shape
-    return lib.lr_select_blocks(ctypes.byref(shape), layer, hq, FAKE, FAKE, FAKE, n_sel, 0.0, blocks, ws,
-                                ws_bytes, None)
+    return lib.lr_select_blocks(ctypes.byref(shape), layer, hq, FAKE, abar, FAKE, n_sel, 0.0, blocks, scores,
+                                ws, ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -151,7 +152,9 @@ def _select(lib, shape=None, layer=0, hq=8, n_sel=4, ws=FAKE, ws_bytes=1 << 40, 
     (dict(blocks=None), lr.LR_ERR_INVALID_ARG),
     (dict(ws=None), lr.LR_ERR_INVALID_ARG),
     (dict(ws_bytes=100), lr.LR_ERR_WORKSPACE),
-    (dict(shape=_shape(rank=16392)), lr.LR_ERR_UNSUPPORTED),
+    (dict(abar=None), lr.LR_ERR_INVALID_ARG),
+    (dict(n_sel=0, abar=None, scores=FAKE), lr.LR_ERR_INVALID_ARG),   # scores asked: Abar needed
+    (dict(scores=FAKE + 4), lr.LR_ERR_INVALID_ARG),                     # misaligned scores_out
 ])
 def test_select_blocks_rejects_bad_arguments(lib, kw, status):
     assert _select(lib, **kw) == status
@@ -165,19 +168,27 @@ def test_select_workspace_counts_queries_and_blocks(lib):
 
 
 def test_decode_path_override_changes_the_plan(lib, monkeypatch):
-    """bf16 / head_dim 128 caches plan the CTA-pair kernel; LOWRAM_DECODE_PATH forces the
-    single-CTA tensor-core or the CUDA-core plan instead (each has its own workspace layout)."""
+    """bf16 / head_dim 128 caches plan the CTA-pair kernel; LOWRAM_DECODE_PATH=general forces
+    the CUDA-core plan instead (it has its own workspace layout)."""
     shape = _shape(T=32768, n_layers=4, n_kv_heads=8, rank=1024)
     sizes = {}
-    for path in ("pair", "tensor", "general"):
+    for path in ("pair", "general"):
         monkeypatch.setenv("LOWRAM_DECODE_PATH", path)
         sizes[path] = lib.lr_decode_workspace_bytes(ctypes.byref(shape), 32, 0)
     monkeypatch.delenv("LOWRAM_DECODE_PATH")
     default = lib.lr_decode_workspace_bytes(ctypes.byref(shape), 32, 0)
     assert default == sizes["pair"]
-    assert len(set(sizes.values())) == 3 and min(sizes.values()) > 0
+    assert len(set(sizes.values())) == 2 and min(sizes.values()) > 0
     f32 = _shape(T=32768, n_layers=4, n_kv_heads=8, rank=1024, dtype=lr.LR_F32)
     monkeypatch.setenv("LOWRAM_DECODE_PATH", "pair")  # not available for fp32: the general plan
     a = lib.lr_decode_workspace_bytes(ctypes.byref(f32), 32, 0)
     monkeypatch.setenv("LOWRAM_DECODE_PATH", "general")
     assert a == lib.lr_decode_workspace_bytes(ctypes.byref(f32), 32, 0)
+
+
+def test_block_means_rejects_bad_arguments(lib):
+    shape = _shape()
+    assert lib.lr_block_means(ctypes.byref(shape), None, FAKE, None) == lr.LR_ERR_INVALID_ARG
+    assert lib.lr_block_means(ctypes.byref(shape), FAKE, FAKE + 8, None) == lr.LR_ERR_INVALID_ARG
+    assert lib.lr_block_means(ctypes.byref(_shape(head_dim=12)), FAKE, FAKE, None) == lr.LR_ERR_UNSUPPORTED
+    assert lib.lr_block_means(ctypes.byref(_shape(T=0)), None, None, None) == lr.LR_OK  # nothing to do

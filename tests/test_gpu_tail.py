@@ -3,7 +3,8 @@ generated tokens in one softmax, against the fp64 oracle on the same inputs.
 
 Cases: a tail next to full and selective reconstruction, a tail with nothing selected
 (the tail alone), a one-token tail alone (the output is that token's value), an empty
-context (T = 0), batch 2, a long tail, the fp32 path and the forced fallback paths.
+context (T = 0), batch 2, a long tail, the fp32 path, the forced CUDA-core path, and the
+262K-token workload (full and 1/16 selective) with a 256-token tail.
 """
 import numpy as np
 import pytest
@@ -95,8 +96,16 @@ def test_tail_fp32_general_path():
     _check(p, 33, rel_l2=1e-4, max_abs=1e-4)
 
 
-@pytest.mark.parametrize("path", ["tensor", "general"])
+@pytest.mark.parametrize("path", ["general"])
 def test_tail_fallback_paths(path, monkeypatch):
     monkeypatch.setenv("LOWRAM_DECODE_PATH", path)
     p = H.packed_problem(H.small(T=900, batch=2), sel=5)
     _check(p, 21)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,sel", [("llama_262k_full", None), ("llama_262k_sel16", "list")])
+def test_tail_full_size(name, sel):
+    w = synth.WORKLOADS[name]
+    p = H.direct_problem(w, sel=w.n_sel if sel else None)
+    _check(p, 256, layer=w.n_layers - 1, blocks=p.blocks)

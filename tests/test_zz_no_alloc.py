@@ -3,9 +3,10 @@ memory (allocator callbacks, runtimes that own every allocation, paths where an 
 may block or fail). It runs on a scratch area compiled into the library instead of a
 caller workspace. This file runs last so that a failure here comes after every other test.
 
-Two calls in a row (different layers, queries and modes) must match the regular entry
-point, which uses its own workspace, within the attention tolerance; a shape whose scratch
-need exceeds the static area is rejected on the host.
+Two calls in a row (different layers, queries and modes) must match the fp64 oracle and the
+regular entry point, which uses its own workspace, within the attention tolerance, and leave
+a clean device error word (read through lr_get_device_error with no workspace); a shape
+whose scratch need exceeds the static area is rejected on the host.
 """
 import ctypes
 
@@ -29,7 +30,7 @@ def _lib():
 
 def _both(p, layer, blocks):
     w = p.w
-    q_st, _ = H.queries(p, layer)
+    q_st, q_ref = H.queries(p, layer)
     shape = H.shape_of(w)
     pred = H.gpu_predictor(p)
     bl = None if blocks is None else torch.from_numpy(np.ascontiguousarray(blocks, dtype=np.int32)).cuda()
@@ -42,14 +43,18 @@ def _both(p, layer, blocks):
     lr.lr_decode_attn_noalloc(shape, layer, w.n_q_heads, q_st, p.st["A"], p.st["Bt"], pred, p.st["idx"],
                               p.st["val"], p.st["ptr"], p.k, bl, n_sel, 0.0, got)
     torch.cuda.synchronize()
-    return got.double().cpu().numpy(), ref.double().cpu().numpy()
+    assert lr.lr_get_device_error(None) == 0
+    want = H.oracle_decode(p, layer, q_ref, blocks=blocks)
+    return got.double().cpu().numpy(), ref.double().cpu().numpy(), want
 
 
-def test_noalloc_matches_regular_entry_on_consecutive_calls():
+def test_noalloc_matches_oracle_and_regular_entry_on_consecutive_calls():
     w = H.small(T=1000, batch=2)
     p = H.packed_problem(w, sel=5)
-    got1, ref1 = _both(p, 1, None)          # full reconstruction
-    got2, ref2 = _both(p, 0, p.blocks)      # selective, the next call on the same scratch
+    got1, ref1, want1 = _both(p, 1, None)          # full reconstruction
+    got2, ref2, want2 = _both(p, 0, p.blocks)      # selective, the next call on the same scratch
+    H.assert_attention_close(got1, want1)
+    H.assert_attention_close(got2, want2)
     H.assert_attention_close(got1, ref1)
     H.assert_attention_close(got2, ref2)
     assert not np.array_equal(got1, got2)
