@@ -9,6 +9,7 @@ a clean device error word (read through lr_get_device_error with no workspace); 
 whose scratch need exceeds the static area is rejected on the host.
 """
 import ctypes
+import dataclasses
 
 import numpy as np
 import pytest
@@ -44,7 +45,8 @@ def _both(p, layer, blocks):
                               p.st["val"], p.st["ptr"], p.k, bl, n_sel, 0.0, got)
     torch.cuda.synchronize()
     assert lr.lr_get_device_error(None) == 0
-    want = H.oracle_decode(p, layer, q_ref, blocks=blocks)
+    # the oracle call names the attended blocks itself (None there means "the problem's list")
+    want = H.oracle_decode(dataclasses.replace(p, blocks=blocks), layer, q_ref)
     return got.double().cpu().numpy(), ref.double().cpu().numpy(), want
 
 
