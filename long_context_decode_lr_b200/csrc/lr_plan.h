@@ -26,11 +26,17 @@ struct DecodePlan {
 };
 
 struct PackPlan {
-  bool tensor;       // tensor-core projection / prediction kernels
+  bool tensor;       // tensor-core projection / key rebuild / predictor kernels
   size_t err_off;    // fp32 errors when the caller passes no err_out
-  size_t diff_off;   // round(v - v_hat) for every token
+  size_t diff_off;   // CUDA-core path: round(v - v_hat) for every token
+  size_t kt_off;     // tensor path: fp16 rebuilt keys K~ [B, T, D]
+  size_t w1h_off;    // tensor path: fp16 copies of W1, W_lin, W2
+  size_t wlh_off;
+  size_t w2h_off;
   size_t ws_bytes;
 };
+
+bool pack_tc_supported(const lr_cache_shape& s);
 
 bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads);
 DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);

@@ -6,6 +6,7 @@
 #include "lr_common.cuh"
 #include "lr_launch.h"
 #include "lr_plan.h"
+#include "lr_gemm.h"
 #include "lr_tc.h"
 
 namespace lr {
@@ -106,14 +107,32 @@ DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm
   return p;
 }
 
+bool pack_tc_supported(const lr_cache_shape& s) {
+  const long long D = (long long)s.n_layers * s.n_kv_heads * s.head_dim;
+  return s.dtype == LR_BF16 && s.head_dim == 128 && (s.hidden == 128 || s.hidden == 256) && s.rank % 128 == 0 &&
+         D % 128 == 0 && s.T > 0;
+}
+
 PackPlan plan_pack(const lr_cache_shape& s, int k) {
   (void)k;
   PackPlan p{};
-  p.tensor = false;
+  const char* env = getenv("LOWRAM_PACK_PATH");
+  p.tensor = pack_tc_supported(s) && !(env && !strcmp(env, "general"));
   const size_t rows = (size_t)s.batch * s.n_layers * s.n_kv_heads * s.T;
   p.err_off = 256;
-  p.diff_off = align256(p.err_off + rows * sizeof(float));
-  p.ws_bytes = align256(p.diff_off + rows * s.head_dim * elem_bytes(s.dtype));
+  const size_t after_err = align256(p.err_off + rows * sizeof(float));
+  if (!p.tensor) {
+    p.diff_off = after_err;
+    p.ws_bytes = align256(p.diff_off + rows * s.head_dim * elem_bytes(s.dtype));
+    return p;
+  }
+  const size_t D = (size_t)s.n_layers * s.n_kv_heads * s.head_dim;
+  const size_t heads = (size_t)s.batch * s.n_layers * s.n_kv_heads;  // per-sequence predictors at most
+  p.kt_off = after_err;
+  p.w1h_off = align256(p.kt_off + (size_t)s.batch * s.T * D * 2);
+  p.wlh_off = align256(p.w1h_off + heads * s.hidden * 128 * 2);
+  p.w2h_off = align256(p.wlh_off + heads * 128 * 128 * 2);
+  p.ws_bytes = align256(p.w2h_off + heads * 128 * s.hidden * 2);
   return p;
 }
 
@@ -170,9 +189,93 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype 
   return launch_decode_combine(a, dt, st);
 }
 
+namespace {
+// The tensor-core pack: projection and key rebuild on the CTA-pair GEMM, the predictor and
+// its error on the fused predictor kernel, the exact top-k, then the residual rows of the
+// kept tokens recomputed by the same predictor kernel in gather mode.
+cudaError_t launch_pack_tc(const PackArgs& a, const PackPlan& plan, cudaStream_t st) {
+  char* ws = (char*)a.errword;
+  void* Kt = ws + plan.kt_off;
+  void* W1h = ws + plan.w1h_off;
+  void* Wlh = ws + plan.wlh_off;
+  void* W2h = ws + plan.w2h_off;
+  const cuuint64_t B = (cuuint64_t)a.B, T = (cuuint64_t)a.T, D = (cuuint64_t)a.D, r = (cuuint64_t)a.r;
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // P1: A = round(K_group . Bt)
+  tc::GemmArgs g1{};
+  g1.B = a.B; g1.M = a.T; g1.N = a.r; g1.K = a.D; g1.bn = a.r % 256 == 0 ? 256 : 128;
+  g1.b_mn_major = true; g1.out_f16 = false; g1.err = a.errword;
+  CUtensorMap mA1, mB1, mC1;
+  {
+    const cuuint64_t dA[3] = {D, T, B}, sA[2] = {D * 2, T * D * 2};
+    const cuuint32_t bA[3] = {64, 128, 1};
+    const cuuint64_t dB[3] = {r, D, B}, sB[2] = {r * 2, D * r * 2};
+    const cuuint32_t bB[3] = {64, 64, 1};
+    const cuuint64_t dC[3] = {r, T, B}, sC[2] = {r * 2, T * r * 2};
+    const cuuint32_t bC[3] = {64, 32, 1};
+    if (!tile_map(&mA1, BF, a.K, 3, dA, sA, bA) || !tile_map(&mB1, BF, a.Bt, 3, dB, sB, bB) ||
+        !tile_map(&mC1, BF, a.A, 3, dC, sC, bC))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = tc::launch_gemm_pair(g1, mA1, mB1, mC1, st);
+  if (e != cudaSuccess) return e;
+  // P2: K~ = A . Bt^T, every (layer, KV head) slice at once, fp16
+  tc::GemmArgs g2{};
+  g2.B = a.B; g2.M = a.T; g2.N = a.D; g2.K = a.r; g2.bn = a.D % 256 == 0 ? 256 : 128;
+  g2.b_mn_major = false; g2.out_f16 = true; g2.err = a.errword;
+  CUtensorMap mA2, mB2, mC2;
+  {
+    const cuuint64_t dA[3] = {r, T, B}, sA[2] = {r * 2, T * r * 2};
+    const cuuint32_t bA[3] = {64, 128, 1};
+    const cuuint64_t dB[3] = {r, D, B}, sB[2] = {r * 2, D * r * 2};
+    const cuuint32_t bB[3] = {64, (cuuint32_t)(g2.bn / 2), 1};
+    const cuuint64_t dC[3] = {D, T, B}, sC[2] = {D * 2, T * D * 2};
+    const cuuint32_t bC[3] = {64, 32, 1};
+    if (!tile_map(&mA2, BF, a.A, 3, dA, sA, bA) || !tile_map(&mB2, BF, a.Bt, 3, dB, sB, bB) ||
+        !tile_map(&mC2, F16, Kt, 3, dC, sC, bC))
+      return cudaErrorInvalidValue;
+  }
+  if ((e = tc::launch_gemm_pair(g2, mA2, mB2, mC2, st)) != cudaSuccess) return e;
+  // fp16 predictor weights
+  const int n_heads = (a.pred_per_seq ? a.B : 1) * a.L * a.Hkv;
+  if ((e = tc::launch_weights_f16(a.W1, a.W_lin, a.W2, n_heads, a.H, W1h, Wlh, W2h, st)) != cudaSuccess) return e;
+  CUtensorMap mKt, mW1, mWl, mW2;
+  {
+    const cuuint64_t dK[3] = {D, T, B}, sK[2] = {D * 2, T * D * 2};
+    const cuuint32_t bK[3] = {64, 128, 1};
+    const cuuint64_t H = (cuuint64_t)a.H, nh = (cuuint64_t)n_heads;
+    const cuuint64_t d1[2] = {128, nh * H}, s1[1] = {256};
+    const cuuint64_t dl[2] = {128, nh * 128}, sl[1] = {256};
+    const cuuint64_t d2[2] = {H, nh * 128}, s2[1] = {H * 2};
+    const cuuint32_t bw[2] = {64, 128};
+    if (!tile_map(&mKt, F16, Kt, 3, dK, sK, bK) || !tile_map(&mW1, F16, W1h, 2, d1, s1, bw) ||
+        !tile_map(&mWl, F16, Wlh, 2, dl, sl, bw) || !tile_map(&mW2, F16, W2h, 2, d2, s2, bw))
+      return cudaErrorInvalidValue;
+  }
+  tc::PredictArgs p{};
+  p.B = a.B; p.T = a.T; p.L = a.L; p.Hkv = a.Hkv; p.H = a.H; p.D = a.D; p.k = a.k;
+  p.pred_per_seq = a.pred_per_seq;
+  p.gather = false;
+  p.Kt = Kt; p.V = a.V; p.b1 = a.b1; p.b2 = a.b2; p.err = a.err;
+  p.res_idx = a.res_idx; p.res_val = a.res_val; p.errword = a.errword;
+  // P3 + P4: predictor and per-token error of every token
+  if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+  // P5: exact top-k per (sequence, layer, KV head)
+  const int n_seg = a.B * a.L * a.Hkv;
+  if ((e = launch_topk(a.err, n_seg, a.T, a.k, a.res_idx, st)) != cudaSuccess) return e;
+  // P6: residual rows of the kept tokens, recomputed; block pointers
+  if (a.k > 0) {
+    p.gather = true;
+    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+  }
+  if (a.res_ptr) return launch_block_ptr(a.res_idx, n_seg, a.k, a.T, a.res_ptr, st);
+  return cudaSuccess;
+}
+}  // namespace
+
 cudaError_t launch_pack(const PackArgs& a, const PackPlan& plan, lr_dtype dt, cudaStream_t st) {
-  (void)plan;
   if (a.T == 0) return launch_block_ptr(a.res_idx, a.res_ptr ? a.B * a.L * a.Hkv : 0, a.k, a.T, a.res_ptr, st);
+  if (plan.tensor) return launch_pack_tc(a, plan, st);
   cudaError_t e = launch_pack_project_general(a, dt, st);
   if (e != cudaSuccess) return e;
   if ((e = launch_pack_predict_general(a, dt, st)) != cudaSuccess) return e;

@@ -192,3 +192,20 @@ def test_block_means_rejects_bad_arguments(lib):
     assert lib.lr_block_means(ctypes.byref(shape), FAKE, FAKE + 8, None) == lr.LR_ERR_INVALID_ARG
     assert lib.lr_block_means(ctypes.byref(_shape(head_dim=12)), FAKE, FAKE, None) == lr.LR_ERR_UNSUPPORTED
     assert lib.lr_block_means(ctypes.byref(_shape(T=0)), None, None, None) == lr.LR_OK  # nothing to do
+
+
+def test_pack_path_override_changes_the_plan(lib, monkeypatch):
+    """bf16 / head_dim 128 caches plan the tensor-core packer (rebuilt-key buffer, fp16
+    weights); LOWRAM_PACK_PATH=general forces the CUDA-core plan (a residual row per token)."""
+    shape = _shape(T=4096, n_layers=4, n_kv_heads=8, rank=1024)
+    monkeypatch.setenv("LOWRAM_PACK_PATH", "general")
+    general = lib.lr_pack_workspace_bytes(ctypes.byref(shape), 409)
+    monkeypatch.delenv("LOWRAM_PACK_PATH")
+    tensor = lib.lr_pack_workspace_bytes(ctypes.byref(shape), 409)
+    D = 4 * 8 * 128
+    assert tensor >= 4096 * D * 2 and general >= 4 * 8 * 4096 * 128 * 2 and tensor != general
+    hd64 = _shape(T=4096, head_dim=64, rank=128)
+    monkeypatch.setenv("LOWRAM_PACK_PATH", "pair")
+    a = lib.lr_pack_workspace_bytes(ctypes.byref(hd64), 409)
+    monkeypatch.setenv("LOWRAM_PACK_PATH", "general")
+    assert a == lib.lr_pack_workspace_bytes(ctypes.byref(hd64), 409)

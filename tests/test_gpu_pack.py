@@ -100,6 +100,9 @@ PACK_CASES = {
     "no_residuals": dict(w=dict(T=640), k=0),
     "every_token": dict(w=dict(T=300), k=300),
     "hd64": dict(w=dict(T=500, head_dim=64, rank=64, hidden=128), k=120),
+    "hidden128": dict(w=dict(T=900, hidden=128), k=90),
+    "rank256_gqa8": dict(w=dict(T=1300, rank=256, q_per_kv=8, n_kv_heads=2), k=260),
+    "one_token": dict(w=dict(T=1, res_pct=100), k=1),
 }
 
 
@@ -166,3 +169,16 @@ def test_pack_full_size(pack_131k, pct):
     g = gpu_pack(p, k)
     band = compare(p, g, k)
     assert band <= 0.001 * k * w.n_layers * w.n_kv_heads
+
+
+# bf16 caches with head_dim 128 and hidden 128 or 256 pack on the tensor cores; the CUDA-core
+# packer serves every other shape. Forcing it on these shapes (LOWRAM_PACK_PATH=general) keeps
+# it under the same parity bar.
+@pytest.mark.parametrize("name", ["ragged_bf16", "batch2_b2", "every_token"])
+def test_pack_general_path(name, monkeypatch):
+    monkeypatch.setenv("LOWRAM_PACK_PATH", "general")
+    c = PACK_CASES[name]
+    w = H.small(**c["w"])
+    p = H.packed_problem(w, k=c["k"], with_b2=c.get("b2", False))
+    g = gpu_pack(p, c["k"])
+    compare(p, g, c["k"])
