@@ -56,7 +56,7 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_work(w: synth.Workload, n_sel: int, n_tail: int = 0):
+def algorithmic_work(w: synth.Workload, n_sel: int, n_tail: int = 0, q2: bool = False):
     """(tensor FLOPs, HBM bytes) one decode step of one layer must do at minimum.
 
     Per attended token and KV head: the key rebuild A.B_l^h (2 r hd FLOPs) and the
@@ -82,7 +82,7 @@ def algorithmic_work(w: synth.Workload, n_sel: int, n_tail: int = 0):
     bytes_ = B * (a_rows * r * e                                  # A rows
                   + Hkv * hd * r * e                              # B_l
                   + Hkv * (hd * hd + 2 * hd * H + H + hd) * e     # predictors
-                  + Hkv * w.k * res_frac * (hd * e + 4)           # residual rows + indices
+                  + Hkv * w.k * res_frac * ((hd // 4 + 8 if q2 else hd * e) + 4)  # residual rows + indices
                   + Hkv * (w.nblk + 1) * 4                        # block pointers
                   + Hkv * n_sel * 4                               # block lists
                   + 2 * Hq * hd * e                               # q and o
@@ -378,11 +378,25 @@ def run_lowram(args, world, rank):
             Kt, Vt = synth.tail_tokens(w, mw, l, n_tail)
             tails.append(tuple(synth.to_storage(x, w.dtype)[0].cuda().contiguous() for x in (Kt, Vt)))
 
+    q2 = args.residuals == "q2"
+    if q2:  # 2-bit residual rows of every copy, quantised on the GPU
+        for c in copies:
+            n_rows = c["val"].numel() // w.head_dim
+            c["codes"] = torch.empty((n_rows, w.head_dim // 4), dtype=torch.uint8, device="cuda")
+            c["lo"] = torch.empty(n_rows, dtype=torch.float32, device="cuda")
+            c["step"] = torch.empty(n_rows, dtype=torch.float32, device="cuda")
+            lr.lr_quantize_residuals(shape, n_rows, c["val"], c["codes"], c["lo"], c["step"])
+            del c["val"]
+        torch.cuda.synchronize()
+
     def step(i, q=None, o=None):
         c = copies[i % n_copies]
         layer = (i // n_copies) % w.n_layers
         qq, oo = c["q"][layer] if q is None else q, outs[i & 1] if o is None else o
-        if n_tail:
+        if q2:
+            lr.lr_decode_attn_q2(shape, layer, w.n_q_heads, qq, c["A"], c["Bt"], c["pred"], c["idx"], c["codes"],
+                                 c["lo"], c["step"], c["ptr"], k, blocks, n_sel, 0.0, oo, ws, stream)
+        elif n_tail:
             lr.lr_decode_attn_tail(shape, layer, w.n_q_heads, qq, c["A"], c["Bt"], c["pred"], c["idx"], c["val"],
                                    c["ptr"], k, blocks, n_sel, tails[layer][0], tails[layer][1], n_tail, 0.0, oo,
                                    ws, stream)
@@ -430,7 +444,7 @@ def run_lowram(args, world, rank):
 
     if rank != 0:
         return None
-    flops, bytes_ = algorithmic_work(w, n_sel, n_tail)
+    flops, bytes_ = algorithmic_work(w, n_sel, n_tail, q2)
     pk, pk_kind = peaks()
     timed_s = ms_total * 1e-3
     tpeak = pk["bf16_tflops_sustained"] if timed_s > 2.0 else pk["bf16_tflops"]
@@ -450,7 +464,7 @@ def run_lowram(args, world, rank):
         "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
         "config": {"workload": w.name, "description": w.description, "batch_per_gpu": w.batch,
                    "context": w.T, "mode": "selective" if n_sel else "full", "n_sel": n_sel,
-                   "residual_pct": w.res_pct, "tail": n_tail,
+                   "residual_pct": w.res_pct, "residuals": "2-bit codes" if q2 else "rows", "tail": n_tail,
                    "step": "one lr_decode_attn call (one layer)" if not n_tail else
                            f"one lr_decode_attn_tail call (one layer, {n_tail} exact tail tokens per KV head)",
                    "l2": f"inputs rotate over {n_copies} device copies of the cache "
@@ -591,11 +605,15 @@ def main():
                     help="workload the packer is timed on (reported under 'pack'); 'none' skips it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--residuals", choices=["rows", "q2"], default="rows",
+                    help="residual rows in the cache dtype, or as 2-bit codes (lr_decode_attn_q2)")
     ap.add_argument("--tail", type=int, default=0,
                     help="exact recent tokens per (sequence, KV head) decoded with the cache (lr_decode_attn_tail)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.tail and args.residuals == "q2":
+        ap.error("--tail and --residuals q2 are separate entry points; pick one")
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -202,6 +202,42 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* shape, int32_t layer, int32_
                               const void* tail_V, int32_t n_tail, float scale, void* o,
                               void* ws, size_t ws_bytes, lr_stream_t stream);
 
+/* ------------------------------------------------------------------ 2-bit residual rows */
+
+/*
+ * lr_quantize_residuals -- store residual rows with 2 bits per number (explainer, comparison
+ * table: LowRAM combined with quantisation keeps 2-bit residuals). The pages name no
+ * quantiser; this one is uniform per row: lo = min, hi = max, step = (hi - lo) / 3, and entry
+ * x gets the code c = nearest integer of (x - lo) / step (ties to the even code), clamped to
+ * 0..3 (code 0 everywhere when step = 0). Each of hi - lo, the step, x - lo and the quotient
+ * is one correctly rounded fp32 operation, so the codes are exact integers of the stored row.
+ * A decode step reads lo + c * step in place of the row (lr_decode_attn_q2).
+ *
+ * Inputs:  res_val [n_rows, hd] in the cache dtype (e.g. the rows lr_pack_prefill wrote,
+ *          n_rows = B * L_g * Hkv * k); shape gives hd (a multiple of 4) and the dtype.
+ * Outputs: res_codes [n_rows, hd / 4] uint8, entry 4i + s in bits 2s..2s+1 of byte i;
+ *          res_lo [n_rows] fp32 row minimum; res_step [n_rows] fp32 level step.
+ * Errors:  shape errors and NULL / misaligned pointers on the host; LR_ERR_CUDA on a launch
+ *          failure. Needs no workspace.
+ */
+lr_status lr_quantize_residuals(const lr_cache_shape* shape, int64_t n_rows, const void* res_val,
+                                uint8_t* res_codes, float* res_lo, float* res_step, lr_stream_t stream);
+
+/*
+ * lr_decode_attn_q2 -- lr_decode_attn over 2-bit residual rows: the residual added to token
+ * t = res_idx[b, l, h, i] is res_lo[b, l, h, i] + c_j * res_step[b, l, h, i] for entry j, c_j
+ * the code of lr_quantize_residuals. Everything else (inputs, output, workspace, errors) is
+ * as lr_decode_attn; res_codes [B, L_g, Hkv, k, hd / 4], res_lo / res_step [B, L_g, Hkv, k]
+ * take the place of res_val (they may be NULL when k == 0).
+ */
+lr_status lr_decode_attn_q2(const lr_cache_shape* shape, int32_t layer, int32_t n_q_heads,
+                            const void* q, const void* A, const void* Bt,
+                            const lr_predictor* predictor, const int32_t* res_idx,
+                            const uint8_t* res_codes, const float* res_lo, const float* res_step,
+                            const int32_t* res_blk_ptr, int32_t k, const int32_t* block_list,
+                            int32_t n_sel, float scale, void* o, void* ws, size_t ws_bytes,
+                            lr_stream_t stream);
+
 /* ------------------------------------------------------------------ block selection */
 
 /*

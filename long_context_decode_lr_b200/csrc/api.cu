@@ -130,8 +130,16 @@ size_t lr_decode_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads, int
 }  // extern "C"
 
 namespace {
+// Residual rows as stored values (res_val) or as 2-bit codes (res_codes, res_lo, res_step).
+struct ResRows {
+  const void* val;
+  const uint8_t* codes;
+  const float* lo;
+  const float* step;
+};
+
 lr_status decode_impl(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q, const void* A,
-                      const void* Bt, const lr_predictor* pred, const int32_t* res_idx, const void* res_val,
+                      const void* Bt, const lr_predictor* pred, const int32_t* res_idx, const ResRows& rr,
                       const int32_t* res_blk_ptr, int32_t k, const int32_t* block_list, int32_t n_sel,
                       const void* tail_K, const void* tail_V, int32_t n_tail, float scale, void* o, void* ws,
                       size_t ws_bytes, lr_stream_t stream) {
@@ -151,7 +159,12 @@ lr_status decode_impl(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads,
   CHECK_PTR(o, "o");
   if (k > 0) {
     CHECK_PTR(res_idx, "res_idx");
-    CHECK_PTR(res_val, "res_val");
+    if (rr.codes) {
+      CHECK_PTR(rr.lo, "res_lo");
+      CHECK_PTR(rr.step, "res_step");
+    } else {
+      CHECK_PTR(rr.val, "res_val");
+    }
   }
   CHECK_OPT_PTR(res_blk_ptr, "res_blk_ptr");
   CHECK_OPT_PTR(block_list, "block_list");
@@ -175,7 +188,8 @@ lr_status decode_impl(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads,
   a.scale = scale > 0.f ? scale : 1.0f / sqrtf((float)s->head_dim);
   a.q = q; a.A = A; a.Bt = Bt;
   a.W_lin = pred->W_lin; a.W1 = pred->W1; a.b1 = pred->b1; a.W2 = pred->W2; a.b2 = pred->b2;
-  a.res_idx = k ? res_idx : nullptr; a.res_val = k ? res_val : nullptr;
+  a.res_idx = k ? res_idx : nullptr; a.res_val = (k && !rr.codes) ? rr.val : nullptr;
+  a.res_codes = k ? rr.codes : nullptr; a.res_lo = k ? rr.lo : nullptr; a.res_step = k ? rr.step : nullptr;
   a.res_ptr = k ? res_blk_ptr : nullptr;
   a.blocks = block_list;
   a.tail_K = n_tail ? tail_K : nullptr;
@@ -198,8 +212,35 @@ lr_status lr_decode_attn(const lr_cache_shape* s, int32_t layer, int32_t n_q_hea
                          const int32_t* res_idx, const void* res_val, const int32_t* res_blk_ptr,
                          int32_t k, const int32_t* block_list, int32_t n_sel, float scale, void* o,
                          void* ws, size_t ws_bytes, lr_stream_t stream) {
-  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, res_val, res_blk_ptr, k, block_list, n_sel,
-                     nullptr, nullptr, 0, scale, o, ws, ws_bytes, stream);
+  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, ResRows{res_val, nullptr, nullptr, nullptr},
+                     res_blk_ptr, k, block_list, n_sel, nullptr, nullptr, 0, scale, o, ws, ws_bytes, stream);
+}
+
+lr_status lr_decode_attn_q2(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
+                            const void* A, const void* Bt, const lr_predictor* pred, const int32_t* res_idx,
+                            const uint8_t* res_codes, const float* res_lo, const float* res_step,
+                            const int32_t* res_blk_ptr, int32_t k, const int32_t* block_list, int32_t n_sel,
+                            float scale, void* o, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  if (s && s->head_dim % 4) return fail(LR_ERR_UNSUPPORTED, "2-bit rows need head_dim % 4 == 0");
+  if (k > 0) CHECK_PTR(res_codes, "res_codes");
+  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, ResRows{nullptr, res_codes, res_lo, res_step},
+                     res_blk_ptr, k, block_list, n_sel, nullptr, nullptr, 0, scale, o, ws, ws_bytes, stream);
+}
+
+lr_status lr_quantize_residuals(const lr_cache_shape* s, int64_t n_rows, const void* res_val, uint8_t* res_codes,
+                                float* res_lo, float* res_step, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (n_rows < 0) return fail(LR_ERR_INVALID_ARG, "n_rows must be >= 0");
+  if (n_rows == 0) return LR_OK;
+  CHECK_PTR(res_val, "res_val");
+  CHECK_PTR(res_codes, "res_codes");
+  CHECK_PTR(res_lo, "res_lo");
+  CHECK_PTR(res_step, "res_step");
+  const cudaError_t e = lr::launch_quantize_rows(res_val, s->dtype, n_rows, s->head_dim, res_codes, res_lo, res_step,
+                                                 (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "residual quantisation launch");
+  return LR_OK;
 }
 
 lr_status lr_decode_attn_tail(const lr_cache_shape* s, int32_t layer, int32_t n_q_heads, const void* q,
@@ -208,8 +249,8 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* s, int32_t layer, int32_t n_
                               int32_t k, const int32_t* block_list, int32_t n_sel, const void* tail_K,
                               const void* tail_V, int32_t n_tail, float scale, void* o, void* ws,
                               size_t ws_bytes, lr_stream_t stream) {
-  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, res_val, res_blk_ptr, k, block_list, n_sel,
-                     tail_K, tail_V, n_tail, scale, o, ws, ws_bytes, stream);
+  return decode_impl(s, layer, n_q_heads, q, A, Bt, pred, res_idx, ResRows{res_val, nullptr, nullptr, nullptr},
+                     res_blk_ptr, k, block_list, n_sel, tail_K, tail_V, n_tail, scale, o, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ block selection

@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(NT) decode_general_kernel(DecodeArgs a) {
   const HeadPredictor<T> P = head_predictor<T>(a, b, a.layer, h);
   const size_t seg = ((size_t)b * a.L + a.layer) * a.Hkv + h;
   const int* ridx = a.k ? a.res_idx + seg * a.k : nullptr;
-  const T* rval = a.k ? (const T*)a.res_val + seg * a.k * hd : nullptr;
+  const size_t seg_row = seg * a.k;
   const int* rptr = (a.k && a.res_ptr) ? a.res_ptr + seg * (a.nblk + 1) : nullptr;
   const T* q = (const T*)a.q + ((size_t)b * Hq + h * G) * hd;
 
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(NT) decode_general_kernel(DecodeArgs a) {
           const int dd = e - hd - H;
           for (int i = e0; i < e1; ++i) {
             const int t = ridx[i] - t0;
-            if (t >= 0 && t < nt) v = fmaf(pg[t], to_f32(rval[(size_t)i * hd + dd]), v);
+            if (t >= 0 && t < nt) v = fmaf(pg[t], residual_entry<T>(a, seg_row, i, dd), v);
           }
         }
         acc[x] = v;

@@ -392,8 +392,10 @@ struct PairEpi {
 // The residual warp of a CTA: for each tile it scatters p_t r_t over the residual rows of
 // the CTA's two blocks ("Predicting the value cache from keys", paragraph 2). Lane l owns
 // dims 4l .. 4l+3; rows of a block are contiguous in res_val (indices ascending), so a batch
-// of 16 rows is one coalesced 256-byte read per row. Loads are issued before waiting for p.
-template <int MG>
+// of 16 rows is one coalesced 256-byte read per row (Q2: 2-bit rows, one 32-byte code read
+// per row, lane l's byte holding its four dims, dequantised as lo + code * step). Loads are
+// issued before waiting for p.
+template <int MG, bool Q2>
 __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* sm, uint64_t* bars,
                                                    volatile int* abort_flag, uint32_t rank, int b, int h, int split,
                                                    int t_begin, int t_end) {
@@ -408,7 +410,8 @@ __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* s
   bool ok = true;
   const size_t seg = ((size_t)b * a.L + a.layer) * a.Hkv + h;
   const int* ridx = a.k > 0 ? a.res_idx + seg * a.k : nullptr;
-  const __nv_bfloat16* rval = a.k > 0 ? a.res_val + seg * a.k * kHd : nullptr;
+  const __nv_bfloat16* rval = (a.k > 0 && !Q2) ? a.res_val + seg * a.k * kHd : nullptr;
+  const size_t segk = seg * a.k;
   const int* rptr = (a.k > 0 && a.res_ptr) ? a.res_ptr + seg * (a.nblk + 1) : nullptr;
   int tl = 0;
   for (int ti = t_begin; ti < t_end && ok; ++ti, ++tl) {
@@ -445,6 +448,7 @@ __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* s
     for (int i0 = 0; i0 < n_tot || !waited; i0 += 16) {
       int tr[16], bh_of[16];
       uint2 rv[16];
+      uint32_t cb[Q2 ? 16 : 1];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int i = i0 + j;
@@ -453,7 +457,13 @@ __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* s
         const bool in = i < n_tot;
         bh_of[j] = bh;
         tr[j] = in ? __ldg(ridx + e) : -1;
-        rv[j] = in ? __ldg(reinterpret_cast<const uint2*>(rval + (size_t)e * kHd) + lane) : make_uint2(0, 0);
+        if (Q2) {
+          cb[j] = in ? (uint32_t)__ldg(a.res_codes + (segk + e) * (kHd / 4) + lane) : 0u;
+          rv[j] = in ? make_uint2(__float_as_uint(__ldg(a.res_lo + segk + e)), __float_as_uint(__ldg(a.res_step + segk + e)))
+                     : make_uint2(0, 0);
+        } else {
+          rv[j] = in ? __ldg(reinterpret_cast<const uint2*>(rval + (size_t)e * kHd) + lane) : make_uint2(0, 0);
+        }
       }
       if (!waited) {
         if (!(ok = __all_sync(0xffffffffu, mbar_wait_cl(&bars[SOFT_DONE], tl & 1, abort_flag)))) break;
@@ -475,9 +485,19 @@ __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* s
           continue;
         }
         const int prow = bh * 64 + (tr[j] - lo[bh]);
-        const __nv_bfloat162 r01 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].x);
-        const __nv_bfloat162 r23 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].y);
-        const float r0 = __low2float(r01), r1 = __high2float(r01), r2 = __low2float(r23), r3 = __high2float(r23);
+        float r0, r1, r2, r3;
+        if (Q2) {
+          const float qlo = __uint_as_float(rv[j].x), qst = __uint_as_float(rv[j].y);
+          const uint32_t c = cb[j];
+          r0 = fmaf((float)(c & 3u), qst, qlo);
+          r1 = fmaf((float)((c >> 2) & 3u), qst, qlo);
+          r2 = fmaf((float)((c >> 4) & 3u), qst, qlo);
+          r3 = fmaf((float)((c >> 6) & 3u), qst, qlo);
+        } else {
+          const __nv_bfloat162 r01 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].x);
+          const __nv_bfloat162 r23 = *reinterpret_cast<const __nv_bfloat162*>(&rv[j].y);
+          r0 = __low2float(r01), r1 = __high2float(r01), r2 = __low2float(r23), r3 = __high2float(r23);
+        }
 #pragma unroll
         for (int g = 0; g < MG; ++g) {
           if (g < G) {
@@ -509,7 +529,7 @@ __device__ __forceinline__ void pair_residual_warp(const PairArgs& a, uint8_t* s
   }
 }
 
-template <int MG>
+template <int MG, bool Q2>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
                    const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapQ,
@@ -735,7 +755,7 @@ decode_pair_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_consta
     }
   } else if (warp == 10) {
     // ---------------------------------------------------------------- residual rows
-    pair_residual_warp<MG>(a, sm, bars, abort_flag, rank, b, h, split, t_begin, t_end);
+    pair_residual_warp<MG, Q2>(a, sm, bars, abort_flag, rank, b, h, split, t_begin, t_end);
   } else {
     // ---------------------------------------------------------------- epilogue (warps 2-9)
     PairEpi<MG> e(a, sm, bars, abort_flag, rank, warp, lane, tmem);
@@ -863,7 +883,7 @@ __global__ void __launch_bounds__(256) decode_pair_prep_kernel(PairArgs a, int n
   if (bits) flag_error(a.err, bits);
 }
 
-template <int MG>
+template <int MG, bool Q2>
 cudaError_t launch_pair_mg(const PairArgs& a, const CUtensorMap& mA, const CUtensorMap& mB0, const CUtensorMap& mB1,
                            const CUtensorMap& mQ, const CUtensorMap& mW1, const int* blocks, int n_sel,
                            cudaStream_t st) {
@@ -884,13 +904,13 @@ cudaError_t launch_pair_mg(const PairArgs& a, const CUtensorMap& mA, const CUten
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, decode_pair_prep_kernel, a, n_w1, n_q, blocks, n_sel);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_pair_kernel<MG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(decode_pair_kernel<MG, Q2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Layout::kSmemBytes);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(2 * a.n_pairs, a.Hkv, a.B);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = Layout::kSmemBytes;
-  e = cudaLaunchKernelEx(&cfg, decode_pair_kernel<MG>, mA, mB0, mB1, mQ, mW1, a);
+  e = cudaLaunchKernelEx(&cfg, decode_pair_kernel<MG, Q2>, mA, mB0, mB1, mQ, mW1, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -902,7 +922,7 @@ int pair_max_clusters() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
   if (cached[dev]) return cached[dev];
-  if (cudaFuncSetAttribute(decode_pair_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(decode_pair_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)Layout::kSmemBytes) != cudaSuccess)
     return 0;
   cudaLaunchConfig_t cfg{};
@@ -917,7 +937,7 @@ int pair_max_clusters() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_pair_kernel<8>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_pair_kernel<8, false>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -928,8 +948,11 @@ int pair_max_clusters() {
 cudaError_t launch_decode_pair(const PairArgs& a, const CUtensorMap& mA, const CUtensorMap& mB0,
                                const CUtensorMap& mB1, const CUtensorMap& mQ, const CUtensorMap& mW1,
                                const int* blocks, int n_sel, cudaStream_t st) {
-  return a.G <= 4 ? launch_pair_mg<4>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st)
-                  : launch_pair_mg<8>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st);
+  if (a.res_codes)
+    return a.G <= 4 ? launch_pair_mg<4, true>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st)
+                    : launch_pair_mg<8, true>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st);
+  return a.G <= 4 ? launch_pair_mg<4, false>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st)
+                  : launch_pair_mg<8, false>(a, mA, mB0, mB1, mQ, mW1, blocks, n_sel, st);
 }
 
 }  // namespace tc

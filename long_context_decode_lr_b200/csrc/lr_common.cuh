@@ -60,7 +60,10 @@ struct DecodeArgs {
   const void* W2;       // [(B,) L, Hkv, hd, H]
   const void* b2;       // [(B,) L, Hkv, hd] or null
   const int* res_idx;   // [B, L, Hkv, k]
-  const void* res_val;  // [B, L, Hkv, k, hd]
+  const void* res_val;  // [B, L, Hkv, k, hd] rows in the cache dtype, or null with 2-bit rows
+  const uint8_t* res_codes;  // 2-bit rows: [B, L, Hkv, k, hd / 4] codes (null otherwise)
+  const float* res_lo;       // 2-bit rows: [B, L, Hkv, k] row minimum
+  const float* res_step;     // 2-bit rows: [B, L, Hkv, k] level step
   const int* res_ptr;   // [B, L, Hkv, nblk + 1] or null
   const int* blocks;    // [B, Hkv, n_sel] or null
   const void* tail_K;   // [B, Hkv, n_tail, hd] exact recent tokens, or null
@@ -72,6 +75,18 @@ struct DecodeArgs {
   int part_stride;      // floats per partial: 4 + hd + H + hd
   int* err;             // device error word
 };
+
+// Entry dd of residual row i of one (sequence, layer, KV head) segment: the stored value, or
+// lo + code * step for 2-bit rows (seg_row = seg * k, the segment's first row).
+template <typename T>
+__device__ __forceinline__ float residual_entry(const DecodeArgs& a, size_t seg_row, int i, int dd) {
+  const size_t row = seg_row + (size_t)i;
+  if (a.res_codes) {
+    const uint32_t byte = a.res_codes[row * (a.hd / 4) + (dd >> 2)];
+    return fmaf((float)((byte >> (2 * (dd & 3))) & 3u), a.res_step[row], a.res_lo[row]);
+  }
+  return to_f32(((const T*)a.res_val)[row * a.hd + dd]);
+}
 
 template <typename T>
 __device__ __forceinline__ HeadPredictor<T> head_predictor(const DecodeArgs& a, int b, int l, int h) {

@@ -23,6 +23,10 @@ cudaError_t launch_pack_project_general(const PackArgs& a, lr_dtype dt, cudaStre
 cudaError_t launch_pack_predict_general(const PackArgs& a, lr_dtype dt, cudaStream_t st);
 cudaError_t launch_pack_gather(const PackArgs& a, lr_dtype dt, cudaStream_t st);
 
+// 2-bit residual rows: codes, row minimum and level step of every row.
+cudaError_t launch_quantize_rows(const void* rows, lr_dtype dt, long long n_rows, int hd, uint8_t* codes, float* lo,
+                                 float* step, cudaStream_t st);
+
 // Top-k token selection (radix select) and residual block pointers.
 cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st);
 cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_out, cudaStream_t st);

@@ -24,7 +24,10 @@ struct PairArgs {
   __half* W1h;                   // workspace: [(B,) Hkv, H, 128] fp16 copy of the layer's W1
   int w1_seqs;                   // 1, or B when each sequence has its own predictor
   const int* res_idx;            // [B, L, Hkv, k]
-  const __nv_bfloat16* res_val;  // [B, L, Hkv, k, 128]
+  const __nv_bfloat16* res_val;  // [B, L, Hkv, k, 128] (null with 2-bit rows)
+  const uint8_t* res_codes;      // 2-bit rows: [B, L, Hkv, k, 32] codes, else null
+  const float* res_lo;           // 2-bit rows: [B, L, Hkv, k] row minimum
+  const float* res_step;         // 2-bit rows: [B, L, Hkv, k] level step
   const int* res_ptr;            // [B, L, Hkv, nblk + 1] or null
   int* sched;                    // selective mode: [B, Hkv, 1 + n_sel] valid blocks; null in full mode
   int sched_stride;              // 1 + n_sel

@@ -153,6 +153,9 @@ cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& plan, lr_dtype 
     t.w1_seqs = a.pred_per_seq ? a.B : 1;
     t.res_idx = a.res_idx;
     t.res_val = (const __nv_bfloat16*)a.res_val;
+    t.res_codes = a.res_codes;
+    t.res_lo = a.res_lo;
+    t.res_step = a.res_step;
     t.res_ptr = a.res_ptr;
     t.sched = a.blocks ? (int*)((char*)a.err + plan.sched_off) : nullptr;
     t.sched_stride = 1 + a.n_sel;

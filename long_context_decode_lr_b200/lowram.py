@@ -70,6 +70,9 @@ def library() -> ctypes.CDLL:
                                          ctypes.c_float, _P, _P, _Z, _P]),
             "lr_select_workspace_bytes": (_Z, [S, _I]),
             "lr_block_means": (_I, [S, _P, _P, _P]),
+            "lr_quantize_residuals": (_I, [S, ctypes.c_int64, _P, _P, _P, _P, _P]),
+            "lr_decode_attn_q2": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _P, _P, _I, _P, _I, ctypes.c_float,
+                                       _P, _P, _Z, _P]),
             "lr_select_blocks": (_I, [S, _I, _I, _P, _P, _P, _I, ctypes.c_float, _P, _P, _P, _Z, _P]),
             "lr_topk_workspace_bytes": (_Z, [_I, _I, _I]),
             "lr_topk_tokens": (_I, [_P, _I, _I, _I, _P, _P, _Z, _P]),
@@ -150,6 +153,22 @@ def lr_decode_attn(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_
         ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
         _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, float(scale),
         _ptr(o), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def lr_quantize_residuals(shape, n_rows, res_val, res_codes, res_lo, res_step, stream=None) -> None:
+    """2-bit codes [n_rows, hd / 4] uint8 plus row minimum and step (fp32) of residual rows."""
+    _check(library().lr_quantize_residuals(ctypes.byref(shape), int(n_rows), _ptr(res_val), _ptr(res_codes),
+                                           _ptr(res_lo), _ptr(res_step), _stream(stream)))
+
+
+def lr_decode_attn_q2(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_idx, res_codes, res_lo,
+                      res_step, res_blk_ptr, k, block_list, n_sel, scale, o, ws, stream=None) -> None:
+    """lr_decode_attn with 2-bit residual rows (codes, row minimum, step)."""
+    _check(library().lr_decode_attn_q2(
+        ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
+        _ptr(res_idx), _ptr(res_codes), _ptr(res_lo), _ptr(res_step), _ptr(res_blk_ptr), k, _ptr(block_list),
+        n_sel, float(scale), _ptr(o), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def lr_decode_attn_noalloc(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_idx, res_val,

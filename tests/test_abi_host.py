@@ -209,3 +209,18 @@ def test_pack_path_override_changes_the_plan(lib, monkeypatch):
     a = lib.lr_pack_workspace_bytes(ctypes.byref(hd64), 409)
     monkeypatch.setenv("LOWRAM_PACK_PATH", "general")
     assert a == lib.lr_pack_workspace_bytes(ctypes.byref(hd64), 409)
+
+
+def test_quantize_and_q2_decode_reject_bad_arguments(lib):
+    shape = _shape()
+    q = lib.lr_quantize_residuals
+    assert q(ctypes.byref(shape), -1, FAKE, FAKE, FAKE, FAKE, None) == lr.LR_ERR_INVALID_ARG
+    assert q(ctypes.byref(shape), 10, None, FAKE, FAKE, FAKE, None) == lr.LR_ERR_INVALID_ARG
+    assert q(ctypes.byref(shape), 10, FAKE, FAKE, None, FAKE, None) == lr.LR_ERR_INVALID_ARG
+    assert q(ctypes.byref(shape), 0, None, None, None, None, None) == lr.LR_OK
+    pred = _pred()
+    d = lib.lr_decode_attn_q2
+    args = lambda codes, lo: (ctypes.byref(shape), 0, 8, FAKE, FAKE, FAKE, ctypes.byref(pred), FAKE, codes, lo, FAKE,
+                              None, 10, None, 0, 0.0, FAKE, FAKE, 1 << 40, None)
+    assert d(*args(None, FAKE)) == lr.LR_ERR_INVALID_ARG
+    assert d(*args(FAKE, None)) == lr.LR_ERR_INVALID_ARG
