@@ -231,7 +231,7 @@ def pack_bytes_per_token(w: synth.Workload) -> float:
     return 2 * w.D * e + w.rank * e + res
 
 
-def time_pack(w: synth.Workload, lr, reps: int = 3):
+def time_pack(w: synth.Workload, lr, reps: int = 3, fit_steps: int = 0):
     """lr_pack_prefill on synthetic keys and values of workload w (basis from the keys'
     population covariance): best of `reps` calls, with its roofline fraction."""
     mw = synth.model_weights(w)
@@ -262,7 +262,9 @@ def time_pack(w: synth.Workload, lr, reps: int = 3):
     code = lr.lr_get_device_error(ws)
     if code:
         raise RuntimeError(f"pack reported device error {code}")
-    del ws, c, A, idx, val, ptr
+    del ws
+    fit = time_fit(w, c, A, shape, lr, fit_steps) if fit_steps else None
+    del c, A, idx, val, ptr
     torch.cuda.empty_cache()
     ms = min(times)
     toks = w.batch * w.T
@@ -276,7 +278,37 @@ def time_pack(w: synth.Workload, lr, reps: int = 3):
     return {"workload": w.name, "ms": ms, "context_tokens_per_s": toks / (ms * 1e-3), "k": k,
             "tflops": tflops, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
             "roofline_ms": t_roof * 1e3, "frac": t_roof / (ms * 1e-3),
-            "peak_source": f"{kind} (burst bf16, HBM copy)", "algorithmic_flops": flops, "algorithmic_bytes": bytes_}
+            "peak_source": f"{kind} (burst bf16, HBM copy)", "algorithmic_flops": flops, "algorithmic_bytes": bytes_,
+            "fit": fit}
+
+
+def time_fit(w: synth.Workload, c, A, shape, lr, n_steps: int):
+    """lr_fit_predictor on the packed context (n_steps of gradient descent from the pinv
+    start), with the per-step roofline: 2 hd (5 H + 2 hd) tensor FLOPs and 4 hd bytes (the
+    rebuilt key and value rows) per token, layer and KV head."""
+    if not lr.lr_fit_workspace_bytes(shape, True):
+        return None
+    f32 = lambda t: t.float().contiguous()
+    params = [f32(c["W_lin"]), f32(c["W1"]), f32(c["b1"]), f32(c["W2"]), None]
+    ws = lr.workspace(lr.lr_fit_workspace_bytes(shape, True))
+    lr.lr_fit_predictor(shape, A, c["Bt"], c["V"], params, 1, 0.0, ws)  # warm-up (lr 0 leaves params)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    lr.lr_fit_predictor(shape, A, c["Bt"], c["V"], params, n_steps, 0.5, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    if lr.lr_get_device_error(ws):
+        raise RuntimeError("fit reported a device error")
+    ms = e0.elapsed_time(e1)
+    units = w.batch * w.T * w.n_layers * w.n_kv_heads * n_steps
+    flops = units * 2 * w.head_dim * (5 * w.hidden + 2 * w.head_dim)
+    bytes_ = units * 4 * w.head_dim
+    pk, kind = peaks()
+    t_roof = max(flops / (pk["bf16_tflops"] * 1e12), bytes_ / (pk["hbm_gbs"] * 1e9))
+    del ws, params
+    return {"steps": n_steps, "ms": ms, "ms_per_step": ms / n_steps, "tflops": flops / (ms * 1e-3) / 1e12,
+            "roofline_ms": t_roof * 1e3, "frac": t_roof / (ms * 1e-3),
+            "note": "includes the one-off key rebuild K~ = A Bt^T before the steps"}
 
 
 def time_select(w: synth.Workload, c, shape, lr, n_sel: int, reps: int = 20):
@@ -352,7 +384,7 @@ def run_lowram(args, world, rank):
     n_sel = w.n_sel
     pack = None
     if rank == 0 and args.pack_workload != "none":
-        pack = time_pack(synth.WORKLOADS[args.pack_workload], lr)
+        pack = time_pack(synth.WORKLOADS[args.pack_workload], lr, fit_steps=args.fit_steps)
     barrier(world)
     c0, shape = decode_cache(w, lr, seed_offset=rank_seed_offset(rank))
     select = time_select(w, c0, shape, lr, n_sel) if (rank == 0 and n_sel) else None
@@ -605,6 +637,8 @@ def main():
                     help="workload the packer is timed on (reported under 'pack'); 'none' skips it")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--fit-steps", type=int, default=4,
+                    help="test-time fitting steps timed on the pack workload (0 skips them)")
     ap.add_argument("--residuals", choices=["rows", "q2"], default="rows",
                     help="residual rows in the cache dtype, or as 2-bit codes (lr_decode_attn_q2)")
     ap.add_argument("--tail", type=int, default=0,

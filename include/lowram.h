@@ -202,6 +202,61 @@ lr_status lr_decode_attn_tail(const lr_cache_shape* shape, int32_t layer, int32_
                               const void* tail_V, int32_t n_tail, float scale, void* o,
                               void* ws, size_t ws_bytes, lr_stream_t stream);
 
+/* ------------------------------------------------------------------ test-time fitting */
+
+/* The predictor's parameters as fp32 arrays (the layouts of lr_predictor), updated in place by
+ * lr_fit_predictor. b2 may be NULL: then the predictor has no b2 and it is not fitted. */
+typedef struct lr_predictor_f32 {
+  float* W_lin;
+  float* W1;
+  float* b1;
+  float* W2;
+  float* b2;
+  int32_t per_sequence;
+} lr_predictor_f32;
+
+/* Copies of the fitted parameters in the cache dtype (the lr_predictor layouts), written after
+ * the last step; b2 may be NULL. */
+typedef struct lr_predictor_out {
+  void* W_lin;
+  void* W1;
+  void* b1;
+  void* W2;
+  void* b2;
+} lr_predictor_out;
+
+/* Workspace bytes lr_fit_predictor needs (0 for a shape it does not support). The answer
+ * depends on the current device's SM count. */
+size_t lr_fit_workspace_bytes(const lr_cache_shape* shape, int32_t per_sequence);
+
+/*
+ * lr_fit_predictor -- test-time fitting of the value predictor to the context's own keys and
+ * values (explainer, paragraph on prefill cost: the per-head network is fitted to each context
+ * with gradient steps, 150 of them in the paper's quick setting, 300 for a full fit; arXiv
+ * abstract: the predictor is fitted at test time). The pages name neither the loss nor the
+ * optimiser; the reading taken is n_steps of full-batch gradient descent
+ *     theta <- theta - lr * grad L(theta),
+ *     L = mean over tokens t and entries j of (v_hat_t[j] - v_t[j])^2,
+ * per (layer, KV head) predictor, over the rebuilt keys k~_t = A[t] . B_l^h and the true values
+ * of the context (of each sequence with per_sequence = 1; of all sequences with 0). theta is
+ * every parameter: W_lin, W1, b1, W2 and b2 when present. GELU is evaluated in the tanh form
+ * of the tensor-core kernels (within 2.71e-4 of x Phi(x)) and its derivative in the same form.
+ * Run it between the projection and the residual selection: lr_pack_prefill with k = 0 gives A,
+ * then this call, then lr_pack_prefill again with the fitted (rounded) predictor.
+ *
+ * Inputs:  A [B, T, r] (cache dtype); Bt [B, D, r]; V [B, L_g, T, Hkv, hd]; params (fp32,
+ *          the starting point: the pseudoinverse initialisation or an earlier fit), updated in
+ *          place; n_steps >= 0; lr >= 0.
+ * Outputs: params; out (or NULL): the fitted parameters rounded to the cache dtype.
+ * Shapes:  bf16 cache, head_dim 128, hidden 128 or 256, rank a multiple of 128
+ *          (LR_ERR_UNSUPPORTED otherwise).
+ * Errors:  host checks before any launch; LR_ERR_CUDA on a launch failure; the workspace's
+ *          error word as for the other calls.
+ */
+lr_status lr_fit_predictor(const lr_cache_shape* shape, const void* A, const void* Bt, const void* V,
+                           const lr_predictor_f32* params, int32_t n_steps, float lr,
+                           const lr_predictor_out* out, void* ws, size_t ws_bytes, lr_stream_t stream);
+
 /* ------------------------------------------------------------------ 2-bit residual rows */
 
 /*

@@ -354,6 +354,61 @@ lr_status lr_pack_prefill(const lr_cache_shape* s, const void* K_group, const vo
   return LR_OK;
 }
 
+// ------------------------------------------------------------------ test-time fitting
+
+size_t lr_fit_workspace_bytes(const lr_cache_shape* s, int32_t per_sequence) {
+  if (check_shape(s) != LR_OK || !lr::pack_tc_supported(*s)) return 0;
+  return lr::plan_fit(*s, per_sequence ? 1 : 0, current_sm_count()).ws_bytes;
+}
+
+lr_status lr_fit_predictor(const lr_cache_shape* s, const void* A, const void* Bt, const void* V,
+                           const lr_predictor_f32* params, int32_t n_steps, float lr,
+                           const lr_predictor_out* out, void* ws, size_t ws_bytes, lr_stream_t stream) {
+  lr_status st = check_shape(s);
+  if (st != LR_OK) return st;
+  if (!lr::pack_tc_supported(*s))
+    return fail(LR_ERR_UNSUPPORTED, "fitting needs a bf16 cache with head_dim 128, hidden 128 or 256, rank %% 128 == 0");
+  if (!params) return fail(LR_ERR_INVALID_ARG, "params is NULL");
+  if (params->per_sequence != 0 && params->per_sequence != 1)
+    return fail(LR_ERR_INVALID_ARG, "params.per_sequence must be 0 or 1");
+  if (n_steps < 0) return fail(LR_ERR_INVALID_ARG, "n_steps must be >= 0");
+  if (!(lr >= 0.f) || lr > 1e30f) return fail(LR_ERR_INVALID_ARG, "lr must be finite and >= 0");
+  CHECK_PTR(A, "A");
+  CHECK_PTR(Bt, "Bt");
+  CHECK_PTR(V, "V");
+  CHECK_PTR(params->W_lin, "params.W_lin");
+  CHECK_PTR(params->W1, "params.W1");
+  CHECK_PTR(params->b1, "params.b1");
+  CHECK_PTR(params->W2, "params.W2");
+  CHECK_OPT_PTR(params->b2, "params.b2");
+  if (out) {
+    CHECK_PTR(out->W_lin, "out.W_lin");
+    CHECK_PTR(out->W1, "out.W1");
+    CHECK_PTR(out->b1, "out.b1");
+    CHECK_PTR(out->W2, "out.W2");
+    CHECK_OPT_PTR(out->b2, "out.b2");
+    if (out->b2 && !params->b2) return fail(LR_ERR_INVALID_ARG, "out.b2 given without params.b2");
+  }
+  const lr::FitPlan plan = lr::plan_fit(*s, params->per_sequence, current_sm_count());
+  if ((st = check_ws(ws, ws_bytes, plan.ws_bytes)) != LR_OK) return st;
+  cudaStream_t cs = (cudaStream_t)stream;
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+  if (s->batch == 0) return LR_OK;
+  lr::FitCall c{};
+  c.A = A; c.Bt = Bt; c.V = V;
+  c.W_lin = params->W_lin; c.W1 = params->W1; c.b1 = params->b1; c.W2 = params->W2; c.b2 = params->b2;
+  c.per_sequence = params->per_sequence;
+  c.n_steps = n_steps;
+  c.lr = lr;
+  if (out) {
+    c.out_Wl = out->W_lin; c.out_W1 = out->W1; c.out_b1 = out->b1; c.out_W2 = out->W2; c.out_b2 = out->b2;
+  }
+  c.ws = ws;
+  if ((e = lr::launch_fit(*s, c, plan, cs)) != cudaSuccess) return cuda_fail(e, "fitting launch");
+  return LR_OK;
+}
+
 // ------------------------------------------------------------------ single steps
 
 size_t lr_topk_workspace_bytes(int32_t n_segments, int32_t T, int32_t k) {

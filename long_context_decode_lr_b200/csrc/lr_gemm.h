@@ -34,6 +34,16 @@ struct PredictArgs {
   int B, T, L, Hkv, H, D, k;
   int pred_per_seq;
   bool gather;
+  // fitting mode (test-time fitting of the predictor): per row R = v_hat - v, g = GELU(u),
+  // dU' = (R W2) * GELU'(u) with u = k~ W1^T + b1; R, g and dU' go to global memory (fp16) for
+  // the gradient contractions, and the biases come from the fp32 master copies
+  bool fit;
+  const float* b1f;      // fit: [(B,) L, Hkv, H] fp32
+  const float* b2f;      // fit: [(B,) L, Hkv, 128] fp32 or null
+  void* Rout;            // fit: [B * L * Hkv, T, 128] fp16
+  void* Gout;            // fit: [B * L * Hkv, T, H] fp16
+  void* DUout;           // fit: [B * L * Hkv, T, H] fp16
+  void* GP;              // fit: per-CTA scratch [grid, 128, H] fp16 (GELU' of the tile's rows)
   const void* Kt;        // [B, T, D] fp16 rebuilt keys of every (layer, KV head)
   const void* V;         // [B, L, T, Hkv, 128] bf16
   const void* b1;        // [(B,) L, Hkv, H] bf16

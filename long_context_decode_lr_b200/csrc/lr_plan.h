@@ -38,6 +38,26 @@ struct PackPlan {
 
 bool pack_tc_supported(const lr_cache_shape& s);
 
+// Test-time fitting: workspace layout and the whole fit (rebuilt keys, then n_steps of
+// forward, gradient and update launches).
+struct FitPlan {
+  size_t kt_off, r_off, g_off, du_off, gp_off, grad_off, w1h_off, wlh_off, w2h_off, ones_off, ws_bytes;
+  int n_wh, gstride, grid;
+};
+FitPlan plan_fit(const lr_cache_shape& s, int per_sequence, int sm_count);
+struct FitCall {
+  const void* A;
+  const void* Bt;
+  const void* V;
+  float *W_lin, *W1, *b1, *W2, *b2;
+  int per_sequence;
+  int n_steps;
+  float lr;
+  void *out_Wl, *out_W1, *out_b1, *out_W2, *out_b2;
+  void* ws;
+};
+cudaError_t launch_fit(const lr_cache_shape& s, const FitCall& c, const FitPlan& plan, cudaStream_t st);
+
 bool decode_pair_supported(const lr_cache_shape& s, int n_q_heads);
 DecodePlan plan_decode(const lr_cache_shape& s, int n_q_heads, int n_sel, int sm_count);
 PackPlan plan_pack(const lr_cache_shape& s, int k);

@@ -11,7 +11,11 @@
 //   normal mode: the per-token error err[seg, t] = sum_j d_j^2 (paragraph 4: tokens are ranked
 //                by this error), for every token of the context;
 //   gather mode: the residual row res_val[seg, i] = round(d) of the tokens t = res_idx[seg, i]
-//                that the top-k step kept, recomputed for those rows only.
+//                that the top-k step kept, recomputed for those rows only;
+//   fit mode:    the pieces of one gradient step of test-time fitting (explainer, paragraph on
+//                prefill cost): R = v_hat - v, g = GELU(u) and, after one more MMA
+//                MMA4 dG = R W2 (M 128, N H, K 128; W2 read MN-major from the same tile),
+//                dU' = dG * GELU'(u), all stored (fp16) for the gradient contractions.
 // Operands are fp16 with fp32 accumulation; GELU is the tanh form fitted to x Phi(x) (within
 // 2.71e-4). A CTA owns a contiguous range of (segment, tile) items; the segment's weights
 // (W1, W_lin, W2 as fp16, 160 KB at H = 256) stay in shared memory while its tiles stream.
@@ -40,13 +44,13 @@ constexpr int kOffKt = 163840;     // k~ tile [atom 0..1][128 rows][128 B]; late
 constexpr int kOffG0 = 196608;     // GELU half 0 [atom 0..1][128 rows][128 B]
 constexpr int kOffEsum = 229376;   // [parity][sub][128] partial errors
 constexpr int kOffBar = 231424;
-constexpr int kOffMisc = kOffBar + 128;
+constexpr int kOffMisc = kOffBar + 192;
 constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum PBar { W_FULL, W_FREE, K_FULL, K_FREE, U_FULL, U_FREE, G_READY0, G_READY1, G0_FREE, V_FULL0, V_FULL1,
-            V_FREE0, V_FREE1, E_READY0, E_READY1, DRAIN, N_PBARS };
-static_assert(N_PBARS * 8 <= 128, "barrier area");
+            V_FREE0, V_FREE1, E_READY0, E_READY1, DRAIN, R_READY, DG_FULL, DG_FREE, N_PBARS };
+static_assert(N_PBARS * 8 <= 192, "barrier area");
 
 constexpr float kGeluC1 = 0.80015708f;  // tanh-form GELU: c1, c3 minimise the largest error
                                         // against x Phi(x) on [-10, 10] (2.71e-4)
@@ -56,6 +60,16 @@ __device__ __forceinline__ float gelu_f32(float x) {
   const float z = x * fmaf(kGeluC3, x * x, kGeluC1);
   const float h = 0.5f * x;
   return fmaf(h, tanh_fast(z), h);
+}
+
+// GELU and its derivative in the same tanh form: with z = x (c1 + c3 x^2) and th = tanh z,
+// GELU = x/2 (1 + th) and GELU' = (1 + th)/2 + x/2 (1 - th^2)(c1 + 3 c3 x^2).
+__device__ __forceinline__ void gelu_and_grad(float x, float& g, float& gp) {
+  const float x2 = x * x;
+  const float th = tanh_fast(x * fmaf(kGeluC3, x2, kGeluC1));
+  const float h = 0.5f * x;
+  g = fmaf(h, th, h);
+  gp = fmaf(0.5f, th, 0.5f) + h * fmaf(-th, th, 1.f) * fmaf(3.f * kGeluC3, x2, kGeluC1);
 }
 
 struct Item {
@@ -131,6 +145,9 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     mbar_init(&bars[E_READY0], 4);
     mbar_init(&bars[E_READY1], 4);
     mbar_init(&bars[DRAIN], 1);
+    mbar_init(&bars[R_READY], 8);
+    mbar_init(&bars[DG_FULL], 1);
+    mbar_init(&bars[DG_FREE], 8);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -235,7 +252,9 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           cur_wh = x.wh;
         }
         if (!(ok = mbar_wait(&bars[K_FULL], i & 1, abort_flag))) break;
-        if (i > 0 && !(ok = mbar_wait(&bars[U_FREE], (i - 1) & 1, abort_flag))) break;
+        // U's columns are free again once the previous tile's GELU read them (fit mode: once
+        // its dG, which reuses them, was read)
+        if (i > 0 && !(ok = mbar_wait(&bars[a.fit ? DG_FREE : U_FREE], (i - 1) & 1, abort_flag))) break;
         if (i >= 2 && !(ok = mbar_wait(&bars[V_FREE0 + (i & 1)], ((i >> 1) - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t vcol = tmem + 256 + 128 * (i & 1);
@@ -256,11 +275,22 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           for (int ks = 0; ks < 8; ++ks)
             mma_f16_ss(vcol, sw128_desc(ga + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                        sw128_desc(w2 + (2 * hf + (ks >> 2)) * 16384 + (ks & 3) * 32, 16, 1024), id_v, 1);
-          if (hf == 0) mma_commit(&bars[G0_FREE]);
+          if (hf == 0 && !a.fit) mma_commit(&bars[G0_FREE]);
         }
         if (!ok) break;
         mma_commit(&bars[V_FULL0 + (i & 1)]);
         mma_commit(&bars[K_FREE]);
+        if (a.fit) {  // MMA4: dG = R W2 with R in the G0 buffer, W2 read MN-major
+          if (!(ok = mbar_wait(&bars[R_READY], i & 1, abort_flag))) break;
+          tc_fence_after();
+          const uint32_t id_dg = idesc_f16_f32(128, H, false, true);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            mma_f16_ss(tmem, sw128_desc(g0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                       sw128_desc(w2 + ks * 2048, 16384, 1024), id_dg, ks != 0);
+          mma_commit(&bars[DG_FULL]);
+          mma_commit(&bars[G0_FREE]);
+        }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -275,10 +305,23 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     const int row = q * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     float* esum = reinterpret_cast<float*>(sm + kOffEsum);
+    __half* gp_row = a.fit ? (__half*)a.GP + ((size_t)blockIdx.x * 128 + row) * H : nullptr;
     bool ok = true;
     for (int it = it0, i = 0; it < it1 && ok; ++it, ++i) {
       const Item x = item_of(a, it, n_t);
+      const int ir = x.tile * 128 + row;
+      // the token of this row: every token (normal and fit modes) or a kept one (gather mode)
+      int t = -1;
+      if (a.gather) {
+        if (ir < a.k) {
+          t = __ldg(a.res_idx + (size_t)x.seg * a.k + ir);
+          if (t < 0 || t >= a.T) t = -1;
+        }
+      } else if (ir < a.T) {
+        t = ir;
+      }
       const __nv_bfloat16* b1 = (const __nv_bfloat16*)a.b1 + (size_t)x.wh * H;
+      const float* b1f = a.fit ? a.b1f + (size_t)x.wh * H : nullptr;
       // ---- GELU branch: this warp's 64 of every 128 hidden units
       if (!(ok = ewait(&bars[U_FULL], i & 1, abort_flag))) break;
       tc_fence_after();
@@ -293,17 +336,41 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         }
         uint8_t* gt = sm + (hf == 0 ? kOffG0 : kOffKt) + sub * 16384 + row * 128;
         if (hf == 0 && i > 0 && !(ok = ewait(&bars[G0_FREE], (i - 1) & 1, abort_flag))) break;
+        const int c0 = hf * 128 + sub * 64;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float bb[8];
-          ld_bf16x8(b1 + hf * 128 + sub * 64 + 8 * j, bb);
+          if (b1f) {
+            const float4 f0 = __ldg(reinterpret_cast<const float4*>(b1f + c0 + 8 * j));
+            const float4 f1 = __ldg(reinterpret_cast<const float4*>(b1f + c0 + 8 * j) + 1);
+            bb[0] = f0.x; bb[1] = f0.y; bb[2] = f0.z; bb[3] = f0.w;
+            bb[4] = f1.x; bb[5] = f1.y; bb[6] = f1.z; bb[7] = f1.w;
+          } else {
+            ld_bf16x8(b1 + c0 + 8 * j, bb);
+          }
           const uint32_t* uu = &u[j >> 2][(j & 3) * 8];
+          float g[8], gp[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float xv = __uint_as_float(uu[c]) + bb[c];
+            if (a.fit) gelu_and_grad(xv, g[c], gp[c]);
+            else g[c] = gelu_f32(xv);
+          }
           uint4 w;
-          w.x = pack_f16x2_sat(gelu_f32(__uint_as_float(uu[0]) + bb[0]), gelu_f32(__uint_as_float(uu[1]) + bb[1]));
-          w.y = pack_f16x2_sat(gelu_f32(__uint_as_float(uu[2]) + bb[2]), gelu_f32(__uint_as_float(uu[3]) + bb[3]));
-          w.z = pack_f16x2_sat(gelu_f32(__uint_as_float(uu[4]) + bb[4]), gelu_f32(__uint_as_float(uu[5]) + bb[5]));
-          w.w = pack_f16x2_sat(gelu_f32(__uint_as_float(uu[6]) + bb[6]), gelu_f32(__uint_as_float(uu[7]) + bb[7]));
+          w.x = pack_f16x2_sat(g[0], g[1]);
+          w.y = pack_f16x2_sat(g[2], g[3]);
+          w.z = pack_f16x2_sat(g[4], g[5]);
+          w.w = pack_f16x2_sat(g[6], g[7]);
           *reinterpret_cast<uint4*>(gt + ((j ^ (row & 7)) << 4)) = w;
+          if (a.fit) {
+            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Gout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
+            uint4 wp;
+            wp.x = pack_f16x2_sat(gp[0], gp[1]);
+            wp.y = pack_f16x2_sat(gp[2], gp[3]);
+            wp.z = pack_f16x2_sat(gp[4], gp[5]);
+            wp.w = pack_f16x2_sat(gp[6], gp[7]);
+            reinterpret_cast<uint4*>(gp_row + c0)[j] = wp;
+          }
         }
         fence_proxy_async_smem();
         warp_arrive(&bars[G_READY0 + hf], lane);
@@ -319,32 +386,29 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       tmem_ld_wait();
       tc_fence_before();
       warp_arrive(&bars[V_FREE0 + par], lane);
-      const int ir = x.tile * 128 + row;
-      int t = -1;
-      if (a.gather) {
-        if (ir < a.k) {
-          t = __ldg(a.res_idx + (size_t)x.seg * a.k + ir);
-          if (t < 0 || t >= a.T) t = -1;
-        }
-      } else if (ir < a.T) {
-        t = ir;
-      }
       float e = 0.f;
-      if (t >= 0) {
+      {
         const __nv_bfloat16* vr = (const __nv_bfloat16*)a.V +
-                                  ((((size_t)x.b * a.L + x.l) * a.T + t) * a.Hkv + x.h) * 128 + sub * 64;
-        const __nv_bfloat16* b2 = a.b2 ? (const __nv_bfloat16*)a.b2 + (size_t)x.wh * 128 + sub * 64 : nullptr;
-        __nv_bfloat16* out = a.gather ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 64 : nullptr;
+                                  ((((size_t)x.b * a.L + x.l) * a.T + (t < 0 ? 0 : t)) * a.Hkv + x.h) * 128 + sub * 64;
+        const __nv_bfloat16* b2 = (!a.fit && a.b2) ? (const __nv_bfloat16*)a.b2 + (size_t)x.wh * 128 + sub * 64 : nullptr;
+        const float* b2f = (a.fit && a.b2f) ? a.b2f + (size_t)x.wh * 128 + sub * 64 : nullptr;
+        __nv_bfloat16* out = (a.gather && t >= 0) ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 64
+                                                  : nullptr;
+        uint8_t* rt = sm + kOffG0 + sub * 16384 + row * 128;  // fit: R as the A operand of MMA4
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float v[8], bb[8];
-          ld_bf16x8(vr + 8 * j, v);
+          if (t >= 0) ld_bf16x8(vr + 8 * j, v);
           if (b2) ld_bf16x8(b2 + 8 * j, bb);
+          if (b2f) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) bb[c] = __ldg(b2f + 8 * j + c);
+          }
           float d[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float p = __uint_as_float(vh[j >> 2][(j & 3) * 8 + c]) + (b2 ? bb[c] : 0.f);
-            d[c] = v[c] - p;
+            const float p = __uint_as_float(vh[j >> 2][(j & 3) * 8 + c]) + ((b2 || b2f) ? bb[c] : 0.f);
+            d[c] = t >= 0 ? v[c] - p : 0.f;
             e = fmaf(d[c], d[c], e);
           }
           if (out) {
@@ -355,9 +419,55 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             w.w = pack_bf16x2(d[6], d[7]);
             reinterpret_cast<uint4*>(out)[j] = w;
           }
+          if (a.fit) {  // R = v_hat - v
+            uint4 w;
+            w.x = pack_f16x2_sat(-d[0], -d[1]);
+            w.y = pack_f16x2_sat(-d[2], -d[3]);
+            w.z = pack_f16x2_sat(-d[4], -d[5]);
+            w.w = pack_f16x2_sat(-d[6], -d[7]);
+            *reinterpret_cast<uint4*>(rt + ((j ^ (row & 7)) << 4)) = w;
+            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Rout + ((size_t)x.seg * a.T + t) * 128 + sub * 64)[j] = w;
+          }
         }
       }
-      if (!a.gather) {
+      if (a.fit) {
+        fence_proxy_async_smem();
+        warp_arrive(&bars[R_READY], lane);
+        // ---- dU' = (R W2) * GELU'(u), this warp's columns of every 128-unit half
+        if (!(ok = ewait(&bars[DG_FULL], i & 1, abort_flag))) break;
+        tc_fence_after();
+        for (int hf = 0; hf < nh; ++hf) {
+          uint32_t dg[2][32];
+          tmem_ld32(trow + hf * 128 + sub * 64, dg[0]);
+          tmem_ld32(trow + hf * 128 + sub * 64 + 32, dg[1]);
+          tmem_ld_wait();
+          if (hf == nh - 1) {
+            tc_fence_before();
+            warp_arrive(&bars[DG_FREE], lane);
+          }
+          const int c0 = hf * 128 + sub * 64;
+          if (t < 0) continue;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 wp = reinterpret_cast<const uint4*>(gp_row + c0)[j];
+            const __half2* hp = reinterpret_cast<const __half2*>(&wp);
+            const uint32_t* gg = &dg[j >> 2][(j & 3) * 8];
+            float du[8];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 f = __half22float2(hp[c]);
+              du[2 * c] = __uint_as_float(gg[2 * c]) * f.x;
+              du[2 * c + 1] = __uint_as_float(gg[2 * c + 1]) * f.y;
+            }
+            uint4 w;
+            w.x = pack_f16x2_sat(du[0], du[1]);
+            w.y = pack_f16x2_sat(du[2], du[3]);
+            w.z = pack_f16x2_sat(du[4], du[5]);
+            w.w = pack_f16x2_sat(du[6], du[7]);
+            reinterpret_cast<uint4*>((__half*)a.DUout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
+          }
+        }
+      } else if (!a.gather) {
         float* es = esum + par * 256;
         if (sub == 1) {
           es[128 + row] = e;

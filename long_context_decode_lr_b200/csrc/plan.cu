@@ -6,6 +6,7 @@
 #include "lr_common.cuh"
 #include "lr_launch.h"
 #include "lr_plan.h"
+#include "lr_fit.h"
 #include "lr_gemm.h"
 #include "lr_tc.h"
 
@@ -275,6 +276,115 @@ cudaError_t launch_pack_tc(const PackArgs& a, const PackPlan& plan, cudaStream_t
   return cudaSuccess;
 }
 }  // namespace
+
+FitPlan plan_fit(const lr_cache_shape& s, int per_sequence, int sm_count) {
+  FitPlan p{};
+  const size_t D = (size_t)s.n_layers * s.n_kv_heads * s.head_dim;
+  const size_t segs = (size_t)s.batch * s.n_layers * s.n_kv_heads;
+  const size_t H = (size_t)s.hidden, T = (size_t)s.T;
+  p.n_wh = (per_sequence ? s.batch : 1) * s.n_layers * s.n_kv_heads;
+  p.gstride = tc::fit_grad_stride(s.hidden);
+  p.grid = sm_count;
+  p.kt_off = 256;
+  p.r_off = align256(p.kt_off + (size_t)s.batch * T * D * 2);
+  p.g_off = align256(p.r_off + segs * T * 128 * 2);
+  p.du_off = align256(p.g_off + segs * T * H * 2);
+  p.gp_off = align256(p.du_off + segs * T * H * 2);
+  p.grad_off = align256(p.gp_off + (size_t)sm_count * 128 * H * 2);
+  p.w1h_off = align256(p.grad_off + (size_t)p.n_wh * p.gstride * 4);
+  p.wlh_off = align256(p.w1h_off + (size_t)p.n_wh * H * 128 * 2);
+  p.w2h_off = align256(p.wlh_off + (size_t)p.n_wh * 128 * 128 * 2);
+  p.ones_off = align256(p.w2h_off + (size_t)p.n_wh * 128 * H * 2);
+  p.ws_bytes = align256(p.ones_off + 64 * 64 * 2);
+  return p;
+}
+
+cudaError_t launch_fit(const lr_cache_shape& s, const FitCall& c, const FitPlan& plan, cudaStream_t st) {
+  char* ws = (char*)c.ws;
+  int* errword = (int*)ws;
+  void* Kt = ws + plan.kt_off;
+  const cuuint64_t B = (cuuint64_t)s.batch, T = (cuuint64_t)s.T, r = (cuuint64_t)s.rank;
+  const cuuint64_t D = (cuuint64_t)s.n_layers * s.n_kv_heads * s.head_dim, H = (cuuint64_t)s.hidden;
+  const cuuint64_t segs = B * s.n_layers * s.n_kv_heads;
+  const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  // rebuilt keys of every (layer, KV head): K~ = A . Bt^T (fp16), once for all steps
+  tc::GemmArgs g2{};
+  g2.B = s.batch; g2.M = s.T; g2.N = (int)D; g2.K = s.rank; g2.bn = D % 256 == 0 ? 256 : 128;
+  g2.b_mn_major = false; g2.out_f16 = true; g2.err = errword;
+  CUtensorMap mA2, mB2, mC2, mKt, mKt64, mW1, mWl, mW2, mR, mDU, mG, mOnes;
+  {
+    const cuuint64_t dA[3] = {r, T, B}, sA[2] = {r * 2, T * r * 2};
+    const cuuint32_t bA[3] = {64, 128, 1};
+    const cuuint64_t dB[3] = {r, D, B}, sB[2] = {r * 2, D * r * 2};
+    const cuuint32_t bB[3] = {64, (cuuint32_t)(g2.bn / 2), 1};
+    const cuuint64_t dK[3] = {D, T, B}, sK[2] = {D * 2, T * D * 2};
+    const cuuint32_t bC[3] = {64, 32, 1}, bK[3] = {64, 128, 1}, b64[3] = {64, 64, 1};
+    const cuuint64_t nh = (cuuint64_t)plan.n_wh;
+    const cuuint64_t d1[2] = {128, nh * H}, s1[1] = {256};
+    const cuuint64_t dl[2] = {128, nh * 128}, sl[1] = {256};
+    const cuuint64_t d2[2] = {H, nh * 128}, s2[1] = {H * 2};
+    const cuuint32_t bw[2] = {64, 128};
+    const cuuint64_t dR[3] = {128, T, segs}, sR[2] = {256, T * 256};
+    const cuuint64_t dU[3] = {H, T, segs}, sU[2] = {H * 2, T * H * 2};
+    const cuuint64_t dO[2] = {64, 64}, sO[1] = {128};
+    const cuuint32_t bO[2] = {64, 64};
+    if (!tile_map(&mA2, BF, c.A, 3, dA, sA, bA) || !tile_map(&mB2, BF, c.Bt, 3, dB, sB, bB) ||
+        !tile_map(&mC2, F16, Kt, 3, dK, sK, bC) || !tile_map(&mKt, F16, Kt, 3, dK, sK, bK) ||
+        !tile_map(&mKt64, F16, Kt, 3, dK, sK, b64) ||
+        !tile_map(&mW1, F16, ws + plan.w1h_off, 2, d1, s1, bw) || !tile_map(&mWl, F16, ws + plan.wlh_off, 2, dl, sl, bw) ||
+        !tile_map(&mW2, F16, ws + plan.w2h_off, 2, d2, s2, bw) ||
+        !tile_map(&mR, F16, ws + plan.r_off, 3, dR, sR, b64) || !tile_map(&mDU, F16, ws + plan.du_off, 3, dU, sU, b64) ||
+        !tile_map(&mG, F16, ws + plan.g_off, 3, dU, sU, b64) || !tile_map(&mOnes, F16, ws + plan.ones_off, 2, dO, sO, bO))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e = tc::launch_gemm_pair(g2, mA2, mB2, mC2, st);
+  if (e != cudaSuccess) return e;
+  if ((e = tc::launch_fit_ones(ws + plan.ones_off, st)) != cudaSuccess) return e;
+  float* grad = (float*)(ws + plan.grad_off);
+  if ((e = cudaMemsetAsync(grad, 0, (size_t)plan.n_wh * plan.gstride * 4, st)) != cudaSuccess) return e;
+  tc::FitUpdateArgs u{};
+  u.n_heads = plan.n_wh; u.H = s.hidden; u.gstride = plan.gstride;
+  u.grad = grad;
+  u.W_lin = c.W_lin; u.W1 = c.W1; u.b1 = c.b1; u.W2 = c.W2; u.b2 = c.b2;
+  u.Wlh = (__half*)(ws + plan.wlh_off); u.W1h = (__half*)(ws + plan.w1h_off); u.W2h = (__half*)(ws + plan.w2h_off);
+  u.out_bf16 = s.dtype == LR_BF16;
+  u.lr = 0.f; u.scale = 0.f;  // fp16 copies of the starting weights only
+  if (c.n_steps == 0) {
+    u.out_Wl = c.out_Wl; u.out_W1 = c.out_W1; u.out_b1 = c.out_b1; u.out_W2 = c.out_W2; u.out_b2 = c.out_b2;
+  }
+  if ((e = tc::launch_fit_update(u, st)) != cudaSuccess) return e;
+  tc::PredictArgs p{};
+  p.B = s.batch; p.T = s.T; p.L = s.n_layers; p.Hkv = s.n_kv_heads; p.H = s.hidden; p.D = (int)D; p.k = 0;
+  p.pred_per_seq = c.per_sequence;
+  p.gather = false;
+  p.fit = true;
+  p.Kt = Kt; p.V = c.V; p.b1 = c.b1; p.b2 = nullptr; p.b1f = c.b1; p.b2f = c.b2;
+  p.Rout = ws + plan.r_off; p.Gout = ws + plan.g_off; p.DUout = ws + plan.du_off; p.GP = ws + plan.gp_off;
+  p.errword = errword;
+  tc::FitGradArgs ga{};
+  ga.B = s.batch; ga.T = s.T; ga.L = s.n_layers; ga.Hkv = s.n_kv_heads; ga.H = s.hidden;
+  ga.pred_per_seq = c.per_sequence; ga.grad = grad; ga.gstride = plan.gstride; ga.errword = errword;
+  {
+    const int nkind = 2 + s.hidden / 128;
+    const long long per_split = (long long)segs * nkind;
+    const int nkc = (s.T + 63) / 64;
+    long long S = (2LL * plan.grid + per_split - 1) / per_split;
+    if (S > nkc) S = nkc;
+    if (S < 1) S = 1;
+    ga.S = (int)S;
+  }
+  u.lr = c.lr;
+  u.scale = 2.0f / ((float)s.T * (c.per_sequence ? 1.0f : (float)s.batch) * (float)s.head_dim);
+  for (int step = 0; step < c.n_steps; ++step) {
+    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+    if ((e = tc::launch_fit_grad(ga, mR, mDU, mG, mKt64, mOnes, st)) != cudaSuccess) return e;
+    if (step == c.n_steps - 1) {
+      u.out_Wl = c.out_Wl; u.out_W1 = c.out_W1; u.out_b1 = c.out_b1; u.out_W2 = c.out_W2; u.out_b2 = c.out_b2;
+    }
+    if ((e = tc::launch_fit_update(u, st)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_pack(const PackArgs& a, const PackPlan& plan, lr_dtype dt, cudaStream_t st) {
   if (a.T == 0) return launch_block_ptr(a.res_idx, a.res_ptr ? a.B * a.L * a.Hkv : 0, a.k, a.T, a.res_ptr, st);

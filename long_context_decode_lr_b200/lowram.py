@@ -43,6 +43,16 @@ class lr_predictor(ctypes.Structure):
                 ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("per_sequence", ctypes.c_int32)]
 
 
+class lr_predictor_f32(ctypes.Structure):
+    _fields_ = [("W_lin", ctypes.c_void_p), ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
+                ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p), ("per_sequence", ctypes.c_int32)]
+
+
+class lr_predictor_out(ctypes.Structure):
+    _fields_ = [("W_lin", ctypes.c_void_p), ("W1", ctypes.c_void_p), ("b1", ctypes.c_void_p),
+                ("W2", ctypes.c_void_p), ("b2", ctypes.c_void_p)]
+
+
 _lib = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int32
@@ -70,6 +80,9 @@ def library() -> ctypes.CDLL:
                                          ctypes.c_float, _P, _P, _Z, _P]),
             "lr_select_workspace_bytes": (_Z, [S, _I]),
             "lr_block_means": (_I, [S, _P, _P, _P]),
+            "lr_fit_workspace_bytes": (_Z, [S, _I]),
+            "lr_fit_predictor": (_I, [S, _P, _P, _P, ctypes.POINTER(lr_predictor_f32), _I, ctypes.c_float,
+                                      ctypes.POINTER(lr_predictor_out), _P, _Z, _P]),
             "lr_quantize_residuals": (_I, [S, ctypes.c_int64, _P, _P, _P, _P, _P]),
             "lr_decode_attn_q2": (_I, [S, _I, _I, _P, _P, _P, Pr, _P, _P, _P, _P, _P, _I, _P, _I, ctypes.c_float,
                                        _P, _P, _Z, _P]),
@@ -153,6 +166,20 @@ def lr_decode_attn(shape, layer, n_q_heads, q, A, Bt, predictor: Predictor, res_
         ctypes.byref(shape), layer, n_q_heads, _ptr(q), _ptr(A), _ptr(Bt), ctypes.byref(predictor.c),
         _ptr(res_idx), _ptr(res_val), _ptr(res_blk_ptr), k, _ptr(block_list), n_sel, float(scale),
         _ptr(o), _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def lr_fit_workspace_bytes(shape: lr_cache_shape, per_sequence: bool = True) -> int:
+    return library().lr_fit_workspace_bytes(ctypes.byref(shape), int(per_sequence))
+
+
+def lr_fit_predictor(shape, A, Bt, V, params, n_steps, lr, ws, out=None, per_sequence=True, stream=None) -> None:
+    """Fit the predictor to the context: params = (W_lin, W1, b1, W2, b2 or None), fp32 tensors
+    updated in place; out = the same five in the cache dtype (written after the last step) or None."""
+    p = lr_predictor_f32(*[_ptr(t) for t in params], int(per_sequence))
+    o = None if out is None else ctypes.byref(lr_predictor_out(*[_ptr(t) for t in out]))
+    _check(library().lr_fit_predictor(ctypes.byref(shape), _ptr(A), _ptr(Bt), _ptr(V), ctypes.byref(p), int(n_steps),
+                                      float(lr), o, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                                      _stream(stream)))
 
 
 def lr_quantize_residuals(shape, n_rows, res_val, res_codes, res_lo, res_step, stream=None) -> None:

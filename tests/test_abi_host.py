@@ -224,3 +224,26 @@ def test_quantize_and_q2_decode_reject_bad_arguments(lib):
                               None, 10, None, 0, 0.0, FAKE, FAKE, 1 << 40, None)
     assert d(*args(None, FAKE)) == lr.LR_ERR_INVALID_ARG
     assert d(*args(FAKE, None)) == lr.LR_ERR_INVALID_ARG
+
+
+def test_fit_predictor_rejects_bad_arguments(lib):
+    shape = _shape()
+    ws_bytes = lib.lr_fit_workspace_bytes(ctypes.byref(shape), 1)
+    assert ws_bytes > 1000 * 2 * 2 * 128 * 2                       # at least the rebuilt keys
+    assert lib.lr_fit_workspace_bytes(ctypes.byref(_shape(head_dim=64)), 1) == 0   # unsupported shape
+    f = lib.lr_fit_predictor
+
+    def call(shape=shape, n_steps=3, step=0.1, b2=None, out=None, ws=FAKE, ws_bytes=ws_bytes, A=FAKE, per_seq=1):
+        p = lr.lr_predictor_f32(FAKE, FAKE, FAKE, FAKE, b2, per_seq)
+        return f(ctypes.byref(shape), A, FAKE, FAKE, ctypes.byref(p), n_steps, step,
+                 None if out is None else ctypes.byref(out), ws, ws_bytes, None)
+
+    assert call(n_steps=-1) == lr.LR_ERR_INVALID_ARG
+    assert call(step=-0.5) == lr.LR_ERR_INVALID_ARG
+    assert call(step=float("nan")) == lr.LR_ERR_INVALID_ARG
+    assert call(A=None) == lr.LR_ERR_INVALID_ARG
+    assert call(per_seq=2) == lr.LR_ERR_INVALID_ARG
+    assert call(ws_bytes=ws_bytes - 1) == lr.LR_ERR_WORKSPACE
+    assert call(shape=_shape(head_dim=64)) == lr.LR_ERR_UNSUPPORTED
+    assert call(shape=_shape(dtype=lr.LR_F32)) == lr.LR_ERR_UNSUPPORTED
+    assert call(out=lr.lr_predictor_out(FAKE, FAKE, FAKE, FAKE, FAKE)) == lr.LR_ERR_INVALID_ARG  # out.b2 w/o b2
