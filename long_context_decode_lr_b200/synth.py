@@ -118,6 +118,9 @@ _add(_mistral("llama_262k_sel16", "Llama-3.1-8B-shaped 4-layer group, B=1, T=262
 for _pct in (5, 10, 25):
     _add(_mistral(f"pack_131k_r{_pct}", f"Mistral-7B-shaped 4-layer group pack, B=1, T=131072, "
                   f"{_pct}% residuals, bf16", 1, 131072, _pct, 0, 1004))
+# a smaller pack of the same shape (inputs still larger than L2), for kernel profiles
+_add(_mistral("pack_32k_r10", "Mistral-7B-shaped 4-layer group pack, B=1, T=32768, 10% residuals, bf16",
+              1, 32768, 10, 0, 1005))
 for _b in (1, 2, 4, 8):
     for _t, _tn in ((32768, "32k"), (131072, "131k")):
         _add(_mistral(f"sweep_b{_b}_{_tn}", f"decode sweep: B={_b}, T={_t}, full reconstruction, "
