@@ -390,6 +390,7 @@ lr_status lr_fit_predictor(const lr_cache_shape* s, const void* A, const void* B
     if (out->b2 && !params->b2) return fail(LR_ERR_INVALID_ARG, "out.b2 given without params.b2");
   }
   const lr::FitPlan plan = lr::plan_fit(*s, params->per_sequence, current_sm_count());
+  if (plan.n_wh > 65535) return fail(LR_ERR_UNSUPPORTED, "more than 65535 predictor heads");
   if ((st = check_ws(ws, ws_bytes, plan.ws_bytes)) != LR_OK) return st;
   cudaStream_t cs = (cudaStream_t)stream;
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, cs);

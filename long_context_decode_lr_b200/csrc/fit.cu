@@ -254,46 +254,34 @@ fit_grad_kernel(const __grid_constant__ CUtensorMap mapR, const __grid_constant_
 
 // theta -= lr * scale * sum for every parameter of every weight head; the sums are cleared and
 // the fp16 copies of W1, W_lin, W2 refreshed (update = 0 with lr = 0: only the copies and the
-// clearing, used before the first step).
+// clearing, used before the first step). One grid row per weight head (blockIdx.y), so each
+// thread's position within the head's parameters needs no division.
+__device__ __forceinline__ void fit_update_one(const FitUpdateArgs& a, float* w, __half* wh16, void* out, size_t o,
+                                               float d) {
+  const float v = w[o] - d;
+  w[o] = v;
+  if (wh16) wh16[o] = __float2half_rn(v);
+  if (out) store_dtype(out, o, v, a.out_bf16);
+}
+
 __global__ void fit_update_kernel(FitUpdateArgs a) {
-  const size_t per = (size_t)a.gstride;
-  const size_t n = (size_t)a.n_heads * per;
+  const size_t wh = blockIdx.y;
   const int H = a.H;
-  for (size_t x = (size_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (size_t)gridDim.x * blockDim.x) {
-    const size_t wh = x / per, e = x % per;
-    const float g = a.grad[x];
-    a.grad[x] = 0.f;
-    const float d = a.lr * a.scale * g;
-    if (e < 128 * 128) {
-      const size_t o = wh * 128 * 128 + e;
-      const float w = a.W_lin[o] - d;
-      a.W_lin[o] = w;
-      a.Wlh[o] = __float2half_rn(w);
-      if (a.out_Wl) store_dtype(a.out_Wl, o, w, a.out_bf16);
-    } else if (e < 128 * 128 + (size_t)H * 128) {
-      const size_t o = wh * H * 128 + (e - 128 * 128);
-      const float w = a.W1[o] - d;
-      a.W1[o] = w;
-      a.W1h[o] = __float2half_rn(w);
-      if (a.out_W1) store_dtype(a.out_W1, o, w, a.out_bf16);
-    } else if (e < 128 * 128 + 2 * (size_t)H * 128) {
-      const size_t o = wh * 128 * H + (e - 128 * 128 - (size_t)H * 128);
-      const float w = a.W2[o] - d;
-      a.W2[o] = w;
-      a.W2h[o] = __float2half_rn(w);
-      if (a.out_W2) store_dtype(a.out_W2, o, w, a.out_bf16);
-    } else if (e < 128 * 128 + 2 * (size_t)H * 128 + H) {
-      const size_t o = wh * H + (e - 128 * 128 - 2 * (size_t)H * 128);
-      const float w = a.b1[o] - d;
-      a.b1[o] = w;
-      if (a.out_b1) store_dtype(a.out_b1, o, w, a.out_bf16);
-    } else {
-      const size_t o = wh * 128 + (e - 128 * 128 - 2 * (size_t)H * 128 - H);
-      if (a.b2) {
-        const float w = a.b2[o] - d;
-        a.b2[o] = w;
-        if (a.out_b2) store_dtype(a.out_b2, o, w, a.out_bf16);
-      }
+  const int n_wl = 128 * 128, n_w1 = H * 128, n_w2 = 128 * H;
+  float* g = a.grad + wh * (size_t)a.gstride;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < a.gstride; e += gridDim.x * blockDim.x) {
+    const float d = a.lr * a.scale * g[e];
+    g[e] = 0.f;
+    if (e < n_wl) {
+      fit_update_one(a, a.W_lin, a.Wlh, a.out_Wl, wh * n_wl + e, d);
+    } else if (e < n_wl + n_w1) {
+      fit_update_one(a, a.W1, a.W1h, a.out_W1, wh * n_w1 + (e - n_wl), d);
+    } else if (e < n_wl + n_w1 + n_w2) {
+      fit_update_one(a, a.W2, a.W2h, a.out_W2, wh * n_w2 + (e - n_wl - n_w1), d);
+    } else if (e < n_wl + n_w1 + n_w2 + H) {
+      fit_update_one(a, a.b1, nullptr, a.out_b1, wh * H + (e - n_wl - n_w1 - n_w2), d);
+    } else if (a.b2) {
+      fit_update_one(a, a.b2, nullptr, a.out_b2, wh * 128 + (e - n_wl - n_w1 - n_w2 - H), d);
     }
   }
 }
@@ -320,10 +308,8 @@ cudaError_t launch_fit_grad(const FitGradArgs& a, const CUtensorMap& mR, const C
 }
 
 cudaError_t launch_fit_update(const FitUpdateArgs& a, cudaStream_t st) {
-  const size_t n = (size_t)a.n_heads * a.gstride;
-  if (n == 0) return cudaSuccess;
-  const int grid = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  fit_update_kernel<<<grid, 256, 0, st>>>(a);
+  if (a.n_heads == 0) return cudaSuccess;
+  fit_update_kernel<<<dim3((a.gstride + 255) / 256, a.n_heads), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -20,8 +20,10 @@
 // 2.71e-4). A CTA owns a contiguous range of (segment, tile) items; the segment's weights
 // (W1, W_lin, W2 as fp16, 160 KB at H = 256) stay in shared memory while its tiles stream.
 // Warp 0 loads (TMA for whole tiles, plain loads for gathered rows), warp 1 issues the MMAs,
-// warps 2-9 are the epilogue (two per TMEM lane quarter, each on half the columns). The
-// second GELU half reuses the k~ buffer, whose readers (MMA2, MMA3a) are done by then.
+// warps 2-9 are the epilogue (two per TMEM lane quarter, each on half the columns). The k~
+// buffer is released as soon as MMA2 and MMA3a have read it, so the next tile's keys load
+// while this tile's GELU halves (one after the other through one fp16 buffer), MMA3b and
+// error run; each epilogue thread starts its value-row loads before it waits for v_hat.
 // Every wait is bounded; a timeout raises the abort flag and sets LR_DEVERR_TIMEOUT.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -40,8 +42,8 @@ constexpr int kThreads = 320;
 constexpr int kOffW1 = 0;          // [k atom 0..1][H rows][128 B]
 constexpr int kOffWl = 65536;      // [k atom 0..1][128 rows][128 B]
 constexpr int kOffW2 = 98304;      // [k atom 0..H/64-1][128 rows][128 B]
-constexpr int kOffKt = 163840;     // k~ tile [atom 0..1][128 rows][128 B]; later the GELU half 1
-constexpr int kOffG0 = 196608;     // GELU half 0 [atom 0..1][128 rows][128 B]
+constexpr int kOffKt = 163840;     // k~ tile [atom 0..1][128 rows][128 B]
+constexpr int kOffG0 = 196608;     // one GELU half at a time (fit mode: then R) [atom 0..1][128 rows][128 B]
 constexpr int kOffEsum = 229376;   // [parity][sub][128] partial errors
 constexpr int kOffBar = 231424;
 constexpr int kOffMisc = kOffBar + 192;
@@ -97,6 +99,26 @@ __device__ __forceinline__ void ld_bf16x8(const __nv_bfloat16* p, float (&v)[8])
     v[2 * i] = f.x;
     v[2 * i + 1] = f.y;
   }
+}
+
+// The token a row of an item reads: every token (normal and fit modes) or a kept one
+// (gather mode); -1 past the end or for an out-of-range index.
+__device__ __forceinline__ int item_token(const PredictArgs& a, const Item& x, int row) {
+  const int ir = x.tile * 128 + row;
+  if (a.gather) {
+    if (ir >= a.k) return -1;
+    const int t = __ldg(a.res_idx + (size_t)x.seg * a.k + ir);
+    return (t < 0 || t >= a.T) ? -1 : t;
+  }
+  return ir < a.T ? ir : -1;
+}
+
+__device__ __forceinline__ const __nv_bfloat16* value_row(const PredictArgs& a, const Item& x, int t, int sub) {
+  return (const __nv_bfloat16*)a.V + ((((size_t)x.b * a.L + x.l) * a.T + (t < 0 ? 0 : t)) * a.Hkv + x.h) * 128 + sub * 64;
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ bool ewait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -267,19 +289,20 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           mma_f16_ss(vcol, sw128_desc(kt + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                      sw128_desc(wl + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024), id_v, ks != 0);
         mma_commit(&bars[U_FULL]);
+        mma_commit(&bars[K_FREE]);  // the keys are read: the next tile's may load
+        // the GELU halves pass through G0 one after the other; G0_FREE completes after every
+        // reader of G0 (nh per tile: after each half but the last, and at the tile's end)
         for (int hf = 0; hf < nh && ok; ++hf) {
           if (!(ok = mbar_wait(&bars[G_READY0 + hf], i & 1, abort_flag))) break;
           tc_fence_after();
-          const uint32_t ga = hf == 0 ? g0 : kt;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
-            mma_f16_ss(vcol, sw128_desc(ga + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+            mma_f16_ss(vcol, sw128_desc(g0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                        sw128_desc(w2 + (2 * hf + (ks >> 2)) * 16384 + (ks & 3) * 32, 16, 1024), id_v, 1);
-          if (hf == 0 && !a.fit) mma_commit(&bars[G0_FREE]);
+          if (hf < nh - 1) mma_commit(&bars[G0_FREE]);
         }
         if (!ok) break;
         mma_commit(&bars[V_FULL0 + (i & 1)]);
-        mma_commit(&bars[K_FREE]);
         if (a.fit) {  // MMA4: dG = R W2 with R in the G0 buffer, W2 read MN-major
           if (!(ok = mbar_wait(&bars[R_READY], i & 1, abort_flag))) break;
           tc_fence_after();
@@ -289,8 +312,8 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             mma_f16_ss(tmem, sw128_desc(g0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
                        sw128_desc(w2 + ks * 2048, 16384, 1024), id_dg, ks != 0);
           mma_commit(&bars[DG_FULL]);
-          mma_commit(&bars[G0_FREE]);
         }
+        mma_commit(&bars[G0_FREE]);
       }
       if (!ok) {
         *abort_flag = 1;
@@ -307,18 +330,19 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     float* esum = reinterpret_cast<float*>(sm + kOffEsum);
     __half* gp_row = a.fit ? (__half*)a.GP + ((size_t)blockIdx.x * 128 + row) * H : nullptr;
     bool ok = true;
+    if (it0 < it1) {  // the first tile's value rows start coming from HBM into L2
+      const Item x0 = item_of(a, it0, n_t);
+      const int t0 = item_token(a, x0, row);
+      if (t0 >= 0) prefetch_l2(value_row(a, x0, t0, sub));
+    }
     for (int it = it0, i = 0; it < it1 && ok; ++it, ++i) {
       const Item x = item_of(a, it, n_t);
       const int ir = x.tile * 128 + row;
-      // the token of this row: every token (normal and fit modes) or a kept one (gather mode)
-      int t = -1;
-      if (a.gather) {
-        if (ir < a.k) {
-          t = __ldg(a.res_idx + (size_t)x.seg * a.k + ir);
-          if (t < 0 || t >= a.T) t = -1;
-        }
-      } else if (ir < a.T) {
-        t = ir;
+      const int t = item_token(a, x, row);
+      if (it + 1 < it1) {  // the next tile's value rows, one tile ahead
+        const Item xn = item_of(a, it + 1, n_t);
+        const int tn = item_token(a, xn, row);
+        if (tn >= 0) prefetch_l2(value_row(a, xn, tn, sub));
       }
       const __nv_bfloat16* b1 = (const __nv_bfloat16*)a.b1 + (size_t)x.wh * H;
       const float* b1f = a.fit ? a.b1f + (size_t)x.wh * H : nullptr;
@@ -326,6 +350,14 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       if (!(ok = ewait(&bars[U_FULL], i & 1, abort_flag))) break;
       tc_fence_after();
       for (int hf = 0; hf < nh && ok; ++hf) {
+        const int c0 = hf * 128 + sub * 64;
+        // this warp's 64 biases (bf16), loaded while the TMEM reads are in flight; with ten
+        // warps per CTA three share an SM sub-partition, which caps a thread at 168 registers
+        uint4 b1raw[8];
+        if (!b1f) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) b1raw[j] = __ldg(reinterpret_cast<const uint4*>(b1 + c0) + j);
+        }
         uint32_t u[2][32];
         tmem_ld32(trow + hf * 128 + sub * 64, u[0]);
         tmem_ld32(trow + hf * 128 + sub * 64 + 32, u[1]);
@@ -334,9 +366,11 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           tc_fence_before();
           warp_arrive(&bars[U_FREE], lane);
         }
-        uint8_t* gt = sm + (hf == 0 ? kOffG0 : kOffKt) + sub * 16384 + row * 128;
-        if (hf == 0 && i > 0 && !(ok = ewait(&bars[G0_FREE], (i - 1) & 1, abort_flag))) break;
-        const int c0 = hf * 128 + sub * 64;
+        uint8_t* gt = sm + kOffG0 + sub * 16384 + row * 128;
+        // G0's previous reader is done: the last MMA of the previous tile (commit i nh - 1),
+        // or MMA3b of half 0 of this tile (commit i nh)
+        const int commit = hf == 0 ? i * nh - 1 : i * nh;
+        if (commit >= 0 && !(ok = ewait(&bars[G0_FREE], commit & 1, abort_flag))) break;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float bb[8];
@@ -346,7 +380,13 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             bb[0] = f0.x; bb[1] = f0.y; bb[2] = f0.z; bb[3] = f0.w;
             bb[4] = f1.x; bb[5] = f1.y; bb[6] = f1.z; bb[7] = f1.w;
           } else {
-            ld_bf16x8(b1 + c0 + 8 * j, bb);
+            const __nv_bfloat162* bp = reinterpret_cast<const __nv_bfloat162*>(&b1raw[j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 f = __bfloat1622float2(bp[c]);
+              bb[2 * c] = f.x;
+              bb[2 * c + 1] = f.y;
+            }
           }
           const uint32_t* uu = &u[j >> 2][(j & 3) * 8];
           float g[8], gp[8];
@@ -376,8 +416,14 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         warp_arrive(&bars[G_READY0 + hf], lane);
       }
       if (!ok) break;
-      // ---- value prediction done: d = v - (v_hat + b2)
+      // ---- value prediction done: d = v - (v_hat + b2); the value row is loaded first
       const int par = i & 1;
+      uint4 vrow[8];
+      {
+        const uint4* vsrc = reinterpret_cast<const uint4*>(value_row(a, x, t, sub));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) vrow[j] = t >= 0 ? __ldg(vsrc + j) : make_uint4(0, 0, 0, 0);
+      }
       if (!(ok = ewait(&bars[V_FULL0 + par], (i >> 1) & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t vh[2][32];
@@ -388,8 +434,6 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       warp_arrive(&bars[V_FREE0 + par], lane);
       float e = 0.f;
       {
-        const __nv_bfloat16* vr = (const __nv_bfloat16*)a.V +
-                                  ((((size_t)x.b * a.L + x.l) * a.T + (t < 0 ? 0 : t)) * a.Hkv + x.h) * 128 + sub * 64;
         const __nv_bfloat16* b2 = (!a.fit && a.b2) ? (const __nv_bfloat16*)a.b2 + (size_t)x.wh * 128 + sub * 64 : nullptr;
         const float* b2f = (a.fit && a.b2f) ? a.b2f + (size_t)x.wh * 128 + sub * 64 : nullptr;
         __nv_bfloat16* out = (a.gather && t >= 0) ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 64
@@ -398,7 +442,15 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float v[8], bb[8];
-          if (t >= 0) ld_bf16x8(vr + 8 * j, v);
+          {
+            const __nv_bfloat162* vp = reinterpret_cast<const __nv_bfloat162*>(&vrow[j]);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float2 f = __bfloat1622float2(vp[c]);
+              v[2 * c] = f.x;
+              v[2 * c + 1] = f.y;
+            }
+          }
           if (b2) ld_bf16x8(b2 + 8 * j, bb);
           if (b2f) {
 #pragma unroll

@@ -11,6 +11,7 @@
 // exact integer work.
 #include "lr_common.cuh"
 #include "lr_launch.h"
+#include "sm100.cuh"
 
 namespace lr {
 namespace {
@@ -123,6 +124,148 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   }
 }
 
+// The same selection for long segments, spread over a cluster of kTkCluster CTAs: CTA r owns
+// the tokens [r * chunk, (r + 1) * chunk). Each radix pass histograms the CTA's tokens, the
+// cluster's histograms are summed through distributed shared memory, and every CTA takes the
+// same digit decision. The compaction then emits each CTA's tokens after those of the CTAs
+// before it (counts exchanged the same way), so the output is ascending and unique as above.
+constexpr int kTkCluster = 8;
+constexpr int TKC_THREADS = 512;
+constexpr int TKC_WARPS = TKC_THREADS / 32;
+
+__device__ __forceinline__ int cta_exclusive_scan(bool flag, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int in_warp = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[warp] = __popc(bal);
+  __syncthreads();
+  int before = 0, sum = 0;
+  for (int w = 0; w < TKC_WARPS; ++w) {
+    const int c = warp_tot[w];
+    if (w < warp) before += c;
+    sum += c;
+  }
+  total = sum;
+  __syncthreads();
+  return before + in_warp;
+}
+
+__global__ void __cluster_dims__(kTkCluster, 1, 1) __launch_bounds__(TKC_THREADS)
+    topk_cluster_kernel(const float* __restrict__ err, int T, int k, int* __restrict__ out_all) {
+  __shared__ int whist[TKC_WARPS][256];
+  __shared__ int hist[256];        // this CTA's histogram (read by the whole cluster)
+  __shared__ int counts[2];        // this CTA's tokens above K* and tied at K* (read by the cluster)
+  __shared__ int sh_digit, sh_kr;
+  __shared__ int warp_tot[TKC_WARPS];
+  const int seg = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = sm100::cluster_cta_rank();
+  const float* e = err + (size_t)seg * T;
+  int* out = out_all + (size_t)seg * k;
+  const int chunk = (T + kTkCluster - 1) / kTkCluster;
+  const int lo = min(T, (int)rank * chunk), hi = min(T, lo + chunk);
+  // k == 0 and k == T are handled on the host side of the launch (every CTA takes this path)
+  uint32_t prefix = 0, mask = 0;
+  int kr = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < TKC_WARPS * 256; i += TKC_THREADS) (&whist[0][0])[i] = 0;
+    __syncthreads();
+    for (int t0 = lo; t0 < hi; t0 += TKC_THREADS) {
+      const int t = t0 + tid;
+      bool act = false;
+      int digit = 0;
+      if (t < hi) {
+        const uint32_t key = order_key(e[t]);
+        act = (key & mask) == prefix;
+        digit = (key >> shift) & 255;
+      }
+      const unsigned actmask = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const unsigned same = __match_any_sync(actmask, digit);
+        if ((__ffs(same) - 1) == lane) atomicAdd(&whist[warp][digit], __popc(same));
+      }
+    }
+    __syncthreads();
+    if (tid < 256) {
+      int s = 0;
+      for (int w = 0; w < TKC_WARPS; ++w) s += whist[w][tid];
+      hist[tid] = s;
+    }
+    sm100::cluster_sync();  // every CTA's histogram is complete
+    if (tid < 256) {
+      int s = 0;
+      for (uint32_t r = 0; r < kTkCluster; ++r) s += (int)sm100::ld_cluster_u32(sm100::mapa_shared(&hist[tid], r));
+      whist[0][tid] = s;  // the cluster's histogram
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int cum = 0, d = 255;
+      for (; d > 0; --d) {
+        if (cum + whist[0][d] >= kr) break;
+        cum += whist[0][d];
+      }
+      sh_digit = d;
+      sh_kr = kr - cum;
+    }
+    sm100::cluster_sync();  // no CTA rewrites its histogram while another still reads it
+    prefix |= (uint32_t)sh_digit << shift;
+    mask |= 255u << shift;
+    kr = sh_kr;
+  }
+  const uint32_t kstar = prefix;
+  const int n_tie = kr;
+  // this CTA's counts above K* and tied at K*
+  int gt = 0, eq = 0;
+  for (int t = lo + tid; t < hi; t += TKC_THREADS) {
+    const uint32_t key = order_key(e[t]);
+    gt += key > kstar;
+    eq += key == kstar;
+  }
+  for (int o = 16; o; o >>= 1) {
+    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+  }
+  if (lane == 0) {
+    whist[0][warp] = gt;
+    whist[1][warp] = eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, q = 0;
+    for (int w = 0; w < TKC_WARPS; ++w) {
+      g += whist[0][w];
+      q += whist[1][w];
+    }
+    counts[0] = g;
+    counts[1] = q;
+  }
+  sm100::cluster_sync();
+  int ties_before = 0, taken_before = 0;
+  for (uint32_t r = 0; r < rank; ++r) {
+    const int g = (int)sm100::ld_cluster_u32(sm100::mapa_shared(&counts[0], r));
+    const int q = (int)sm100::ld_cluster_u32(sm100::mapa_shared(&counts[1], r));
+    const int tie_take = max(0, min(q, n_tie - ties_before));
+    taken_before += g + tie_take;
+    ties_before += q;
+  }
+  sm100::cluster_sync();  // every CTA has read the counts it needs before any CTA may exit
+  for (int t0 = lo; t0 < hi; t0 += TKC_THREADS) {
+    const int t = t0 + tid;
+    uint32_t key = 0;
+    const bool valid = t < hi;
+    if (valid) key = order_key(e[t]);
+    const bool is_eq = valid && key == kstar;
+    int eq_total;
+    const int eq_rank = ties_before + cta_exclusive_scan(is_eq, warp_tot, eq_total);
+    const bool take = valid && (key > kstar || (is_eq && eq_rank < n_tie));
+    int take_total;
+    const int pos = taken_before + cta_exclusive_scan(take, warp_tot, take_total);
+    if (take) out[pos] = t;
+    ties_before += eq_total;
+    taken_before += take_total;
+  }
+}
+
 __global__ void block_ptr_kernel(const int* __restrict__ idx, int n_seg, int k, int T, int nblk,
                                  int* __restrict__ ptr) {
   const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -142,6 +285,10 @@ __global__ void block_ptr_kernel(const int* __restrict__ idx, int n_seg, int k, 
 
 cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st) {
   if (n_seg == 0 || k == 0) return cudaSuccess;
+  if (T >= 16384 && k < T) {  // long segments: one cluster of CTAs per segment
+    topk_cluster_kernel<<<dim3(kTkCluster, n_seg), TKC_THREADS, 0, st>>>(err, T, k, idx_out);
+    return cudaGetLastError();
+  }
   topk_kernel<<<n_seg, TK_THREADS, 0, st>>>(err, T, k, idx_out);
   return cudaGetLastError();
 }
