@@ -20,7 +20,8 @@
 // 2.71e-4). A CTA owns a contiguous range of (segment, tile) items; the segment's weights
 // (W1, W_lin, W2 as fp16, 160 KB at H = 256) stay in shared memory while its tiles stream.
 // Warp 0 loads (TMA for whole tiles, plain loads for gathered rows), warp 1 issues the MMAs,
-// warps 2-9 are the epilogue (two per TMEM lane quarter, each on half the columns). The k~
+// warps 2-17 are the epilogue (four per TMEM lane quarter, each on a quarter of the columns
+// of every 128-column half: with eighteen warps a thread keeps at most 104 registers). The k~
 // buffer is released as soon as MMA2 and MMA3a have read it, so the next tile's keys load
 // while this tile's GELU halves (one after the other through one fp16 buffer), MMA3b and
 // error run; each epilogue thread starts its value-row loads before it waits for v_hat.
@@ -38,13 +39,14 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
+constexpr int kEpiWarps = 16;                // four per TMEM lane quarter, 32 columns each
+constexpr int kThreads = 32 * (2 + kEpiWarps);
 constexpr int kOffW1 = 0;          // [k atom 0..1][H rows][128 B]
 constexpr int kOffWl = 65536;      // [k atom 0..1][128 rows][128 B]
 constexpr int kOffW2 = 98304;      // [k atom 0..H/64-1][128 rows][128 B]
 constexpr int kOffKt = 163840;     // k~ tile [atom 0..1][128 rows][128 B]
 constexpr int kOffG0 = 196608;     // one GELU half at a time (fit mode: then R) [atom 0..1][128 rows][128 B]
-constexpr int kOffEsum = 229376;   // [parity][sub][128] partial errors
+constexpr int kOffEsum = 229376;   // [sub 1..3][128] partial errors (sub 0 adds them)
 constexpr int kOffBar = 231424;
 constexpr int kOffMisc = kOffBar + 192;
 constexpr int kSmemBytes = kOffMisc + 64;
@@ -103,9 +105,10 @@ __device__ __forceinline__ void ld_bf16x8(const __nv_bfloat16* p, float (&v)[8])
 
 // The token a row of an item reads: every token (normal and fit modes) or a kept one
 // (gather mode); -1 past the end or for an out-of-range index.
+template <bool kGather>
 __device__ __forceinline__ int item_token(const PredictArgs& a, const Item& x, int row) {
   const int ir = x.tile * 128 + row;
-  if (a.gather) {
+  if (kGather) {
     if (ir >= a.k) return -1;
     const int t = __ldg(a.res_idx + (size_t)x.seg * a.k + ir);
     return (t < 0 || t >= a.T) ? -1 : t;
@@ -114,7 +117,7 @@ __device__ __forceinline__ int item_token(const PredictArgs& a, const Item& x, i
 }
 
 __device__ __forceinline__ const __nv_bfloat16* value_row(const PredictArgs& a, const Item& x, int t, int sub) {
-  return (const __nv_bfloat16*)a.V + ((((size_t)x.b * a.L + x.l) * a.T + (t < 0 ? 0 : t)) * a.Hkv + x.h) * 128 + sub * 64;
+  return (const __nv_bfloat16*)a.V + ((((size_t)x.b * a.L + x.l) * a.T + (t < 0 ? 0 : t)) * a.Hkv + x.h) * 128 + sub * 32;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
@@ -130,10 +133,12 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
+template <int kMode>  // 0 error of every token, 1 residual rows of the kept tokens, 2 fitting step
 __global__ void __launch_bounds__(kThreads, 1)
 pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_constant__ CUtensorMap mapW1,
                        const __grid_constant__ CUtensorMap mapWl, const __grid_constant__ CUtensorMap mapW2,
                        const PredictArgs a) {
+  constexpr bool kGather = kMode == 1, kFit = kMode == 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw;
   if (smem_u32(sm) & 1023u) {
@@ -145,7 +150,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + kOffMisc + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = a.H, nh = a.H / 128;
-  const int n_t = a.gather ? (a.k + 127) / 128 : (a.T + 127) / 128;
+  const int n_t = kGather ? (a.k + 127) / 128 : (a.T + 127) / 128;
   const int n_items = a.B * a.L * a.Hkv * n_t;
   const int it0 = (int)((long long)blockIdx.x * n_items / gridDim.x);
   const int it1 = (int)((long long)(blockIdx.x + 1) * n_items / gridDim.x);
@@ -156,20 +161,20 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     mbar_init(&bars[K_FULL], 1);
     mbar_init(&bars[K_FREE], 1);
     mbar_init(&bars[U_FULL], 1);
-    mbar_init(&bars[U_FREE], 8);
-    mbar_init(&bars[G_READY0], 8);
-    mbar_init(&bars[G_READY1], 8);
+    mbar_init(&bars[U_FREE], kEpiWarps);
+    mbar_init(&bars[G_READY0], kEpiWarps);
+    mbar_init(&bars[G_READY1], kEpiWarps);
     mbar_init(&bars[G0_FREE], 1);
     mbar_init(&bars[V_FULL0], 1);
     mbar_init(&bars[V_FULL1], 1);
-    mbar_init(&bars[V_FREE0], 8);
-    mbar_init(&bars[V_FREE1], 8);
-    mbar_init(&bars[E_READY0], 4);
-    mbar_init(&bars[E_READY1], 4);
+    mbar_init(&bars[V_FREE0], kEpiWarps);
+    mbar_init(&bars[V_FREE1], kEpiWarps);
+    mbar_init(&bars[E_READY0], 12);  // the warps of subs 1-3
+    mbar_init(&bars[E_READY1], 12);
     mbar_init(&bars[DRAIN], 1);
-    mbar_init(&bars[R_READY], 8);
+    mbar_init(&bars[R_READY], kEpiWarps);
     mbar_init(&bars[DG_FULL], 1);
-    mbar_init(&bars[DG_FREE], 8);
+    mbar_init(&bars[DG_FREE], kEpiWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -213,7 +218,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       }
       if (i > 0 && !(ok = ewait(&bars[K_FREE], (i - 1) & 1, abort_flag))) break;
       const int col0 = (x.l * a.Hkv + x.h) * 128;
-      if (!a.gather) {
+      if (!kGather) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&bars[K_FULL], 32768u);
           tma_load_3d(sm + kOffKt, &mapKt, &bars[K_FULL], col0, x.tile * 128, x.b);
@@ -236,12 +241,17 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           }
           const uint4* src = reinterpret_cast<const uint4*>(
               (const __half*)a.Kt + ((size_t)x.b * a.T + (t < 0 ? 0 : t)) * a.D + col0);
-          uint4 v[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) v[c] = t >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+          for (int h4 = 0; h4 < 4; ++h4) {  // half a 64-column atom at a time
+            uint4 v[4];
 #pragma unroll
-          for (int c = 0; c < 16; ++c)
-            *reinterpret_cast<uint4*>(sm + kOffKt + (c >> 3) * 16384 + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v[c];
+            for (int c = 0; c < 4; ++c) v[c] = t >= 0 ? __ldg(src + 4 * h4 + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int q16 = 4 * (h4 & 1) + c;
+              *reinterpret_cast<uint4*>(sm + kOffKt + (h4 >> 1) * 16384 + row * 128 + ((q16 ^ (row & 7)) << 4)) = v[c];
+            }
+          }
         }
         if (bad) flag_error(a.errword, bad);
         fence_proxy_async_smem();
@@ -276,7 +286,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         if (!(ok = mbar_wait(&bars[K_FULL], i & 1, abort_flag))) break;
         // U's columns are free again once the previous tile's GELU read them (fit mode: once
         // its dG, which reuses them, was read)
-        if (i > 0 && !(ok = mbar_wait(&bars[a.fit ? DG_FREE : U_FREE], (i - 1) & 1, abort_flag))) break;
+        if (i > 0 && !(ok = mbar_wait(&bars[kFit ? DG_FREE : U_FREE], (i - 1) & 1, abort_flag))) break;
         if (i >= 2 && !(ok = mbar_wait(&bars[V_FREE0 + (i & 1)], ((i >> 1) - 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t vcol = tmem + 256 + 128 * (i & 1);
@@ -303,7 +313,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         }
         if (!ok) break;
         mma_commit(&bars[V_FULL0 + (i & 1)]);
-        if (a.fit) {  // MMA4: dG = R W2 with R in the G0 buffer, W2 read MN-major
+        if (kFit) {  // MMA4: dG = R W2 with R in the G0 buffer, W2 read MN-major
           if (!(ok = mbar_wait(&bars[R_READY], i & 1, abort_flag))) break;
           tc_fence_after();
           const uint32_t id_dg = idesc_f16_f32(128, H, false, true);
@@ -323,56 +333,54 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       mbar_wait_drain(&bars[DRAIN], 0, kWaitCycles / 4);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2-9)
-    const int q = warp & 3, sub = (warp - 2) >> 2;
+    // ---------------------------------------------------------------- epilogue (warps 2-17)
+    const int q = warp & 3, sub = (warp - 2) >> 2;  // lane quarter, 32-column slice
     const int row = q * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     float* esum = reinterpret_cast<float*>(sm + kOffEsum);
-    __half* gp_row = a.fit ? (__half*)a.GP + ((size_t)blockIdx.x * 128 + row) * H : nullptr;
+    __half* gp_row = kFit ? (__half*)a.GP + ((size_t)blockIdx.x * 128 + row) * H : nullptr;
     bool ok = true;
     if (it0 < it1) {  // the first tile's value rows start coming from HBM into L2
       const Item x0 = item_of(a, it0, n_t);
-      const int t0 = item_token(a, x0, row);
+      const int t0 = item_token<kGather>(a, x0, row);
       if (t0 >= 0) prefetch_l2(value_row(a, x0, t0, sub));
     }
     for (int it = it0, i = 0; it < it1 && ok; ++it, ++i) {
       const Item x = item_of(a, it, n_t);
       const int ir = x.tile * 128 + row;
-      const int t = item_token(a, x, row);
+      const int t = item_token<kGather>(a, x, row);
       if (it + 1 < it1) {  // the next tile's value rows, one tile ahead
         const Item xn = item_of(a, it + 1, n_t);
-        const int tn = item_token(a, xn, row);
+        const int tn = item_token<kGather>(a, xn, row);
         if (tn >= 0) prefetch_l2(value_row(a, xn, tn, sub));
       }
       const __nv_bfloat16* b1 = (const __nv_bfloat16*)a.b1 + (size_t)x.wh * H;
-      const float* b1f = a.fit ? a.b1f + (size_t)x.wh * H : nullptr;
+      const float* b1f = kFit ? a.b1f + (size_t)x.wh * H : nullptr;
       // ---- GELU branch: this warp's 64 of every 128 hidden units
       if (!(ok = ewait(&bars[U_FULL], i & 1, abort_flag))) break;
       tc_fence_after();
+      // this warp's 32 of every 128 hidden units
       for (int hf = 0; hf < nh && ok; ++hf) {
-        const int c0 = hf * 128 + sub * 64;
-        // this warp's 64 biases (bf16), loaded while the TMEM reads are in flight; with ten
-        // warps per CTA three share an SM sub-partition, which caps a thread at 168 registers
-        uint4 b1raw[8];
+        const int c0 = hf * 128 + sub * 32;
+        uint8_t* gt = sm + kOffG0 + (sub >> 1) * 16384 + row * 128;  // atom sub/2, chunks 4(sub&1)..+3
+        uint4 b1raw[4];  // bf16 biases, loaded while the TMEM read is in flight
         if (!b1f) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) b1raw[j] = __ldg(reinterpret_cast<const uint4*>(b1 + c0) + j);
+          for (int j = 0; j < 4; ++j) b1raw[j] = __ldg(reinterpret_cast<const uint4*>(b1 + c0) + j);
         }
-        uint32_t u[2][32];
-        tmem_ld32(trow + hf * 128 + sub * 64, u[0]);
-        tmem_ld32(trow + hf * 128 + sub * 64 + 32, u[1]);
+        uint32_t u[32];
+        tmem_ld32(trow + c0, u);
         tmem_ld_wait();
         if (hf == nh - 1) {
           tc_fence_before();
           warp_arrive(&bars[U_FREE], lane);
         }
-        uint8_t* gt = sm + kOffG0 + sub * 16384 + row * 128;
-        // G0's previous reader is done: the last MMA of the previous tile (commit i nh - 1),
-        // or MMA3b of half 0 of this tile (commit i nh)
+        // G0's previous reader is done: the last MMA of the previous tile (commit i nh - 1), or
+        // MMA3b of half 0 of this tile (commit i nh)
         const int commit = hf == 0 ? i * nh - 1 : i * nh;
         if (commit >= 0 && !(ok = ewait(&bars[G0_FREE], commit & 1, abort_flag))) break;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           float bb[8];
           if (b1f) {
             const float4 f0 = __ldg(reinterpret_cast<const float4*>(b1f + c0 + 8 * j));
@@ -388,12 +396,11 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
               bb[2 * c + 1] = f.y;
             }
           }
-          const uint32_t* uu = &u[j >> 2][(j & 3) * 8];
           float g[8], gp[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float xv = __uint_as_float(uu[c]) + bb[c];
-            if (a.fit) gelu_and_grad(xv, g[c], gp[c]);
+            const float xv = __uint_as_float(u[8 * j + c]) + bb[c];
+            if (kFit) gelu_and_grad(xv, g[c], gp[c]);
             else g[c] = gelu_f32(xv);
           }
           uint4 w;
@@ -401,8 +408,9 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           w.y = pack_f16x2_sat(g[2], g[3]);
           w.z = pack_f16x2_sat(g[4], g[5]);
           w.w = pack_f16x2_sat(g[6], g[7]);
-          *reinterpret_cast<uint4*>(gt + ((j ^ (row & 7)) << 4)) = w;
-          if (a.fit) {
+          const int q16 = 4 * (sub & 1) + j;  // 16-byte chunk of the row within the atom
+          *reinterpret_cast<uint4*>(gt + ((q16 ^ (row & 7)) << 4)) = w;
+          if (kFit) {
             if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Gout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
             uint4 wp;
             wp.x = pack_f16x2_sat(gp[0], gp[1]);
@@ -418,29 +426,28 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       if (!ok) break;
       // ---- value prediction done: d = v - (v_hat + b2); the value row is loaded first
       const int par = i & 1;
-      uint4 vrow[8];
+      uint4 vrow[4];
       {
         const uint4* vsrc = reinterpret_cast<const uint4*>(value_row(a, x, t, sub));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) vrow[j] = t >= 0 ? __ldg(vsrc + j) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < 4; ++j) vrow[j] = t >= 0 ? __ldg(vsrc + j) : make_uint4(0, 0, 0, 0);
       }
       if (!(ok = ewait(&bars[V_FULL0 + par], (i >> 1) & 1, abort_flag))) break;
       tc_fence_after();
-      uint32_t vh[2][32];
-      tmem_ld32(trow + 256 + 128 * par + sub * 64, vh[0]);
-      tmem_ld32(trow + 256 + 128 * par + sub * 64 + 32, vh[1]);
-      tmem_ld_wait();
-      tc_fence_before();
-      warp_arrive(&bars[V_FREE0 + par], lane);
       float e = 0.f;
       {
-        const __nv_bfloat16* b2 = (!a.fit && a.b2) ? (const __nv_bfloat16*)a.b2 + (size_t)x.wh * 128 + sub * 64 : nullptr;
-        const float* b2f = (a.fit && a.b2f) ? a.b2f + (size_t)x.wh * 128 + sub * 64 : nullptr;
-        __nv_bfloat16* out = (a.gather && t >= 0) ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 64
+        const __nv_bfloat16* b2 = (!kFit && a.b2) ? (const __nv_bfloat16*)a.b2 + (size_t)x.wh * 128 + sub * 32 : nullptr;
+        const float* b2f = (kFit && a.b2f) ? a.b2f + (size_t)x.wh * 128 + sub * 32 : nullptr;
+        __nv_bfloat16* out = (kGather && t >= 0) ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 32
                                                   : nullptr;
-        uint8_t* rt = sm + kOffG0 + sub * 16384 + row * 128;  // fit: R as the A operand of MMA4
+        uint8_t* rt = sm + kOffG0 + (sub >> 1) * 16384 + row * 128;  // fit: R as the A operand of MMA4
+        uint32_t vh[32];
+        tmem_ld32(trow + 256 + 128 * par + sub * 32, vh);
+        tmem_ld_wait();
+        tc_fence_before();
+        warp_arrive(&bars[V_FREE0 + par], lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
           float v[8], bb[8];
           {
             const __nv_bfloat162* vp = reinterpret_cast<const __nv_bfloat162*>(&vrow[j]);
@@ -459,7 +466,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           float d[8];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
-            const float p = __uint_as_float(vh[j >> 2][(j & 3) * 8 + c]) + ((b2 || b2f) ? bb[c] : 0.f);
+            const float p = __uint_as_float(vh[8 * j + c]) + ((b2 || b2f) ? bb[c] : 0.f);
             d[c] = t >= 0 ? v[c] - p : 0.f;
             e = fmaf(d[c], d[c], e);
           }
@@ -471,39 +478,39 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             w.w = pack_bf16x2(d[6], d[7]);
             reinterpret_cast<uint4*>(out)[j] = w;
           }
-          if (a.fit) {  // R = v_hat - v
+          if (kFit) {  // R = v_hat - v
             uint4 w;
             w.x = pack_f16x2_sat(-d[0], -d[1]);
             w.y = pack_f16x2_sat(-d[2], -d[3]);
             w.z = pack_f16x2_sat(-d[4], -d[5]);
             w.w = pack_f16x2_sat(-d[6], -d[7]);
-            *reinterpret_cast<uint4*>(rt + ((j ^ (row & 7)) << 4)) = w;
-            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Rout + ((size_t)x.seg * a.T + t) * 128 + sub * 64)[j] = w;
+            const int q16 = 4 * (sub & 1) + j;
+            *reinterpret_cast<uint4*>(rt + ((q16 ^ (row & 7)) << 4)) = w;
+            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Rout + ((size_t)x.seg * a.T + t) * 128 + sub * 32)[j] = w;
           }
         }
       }
-      if (a.fit) {
+      if (kFit) {
         fence_proxy_async_smem();
         warp_arrive(&bars[R_READY], lane);
         // ---- dU' = (R W2) * GELU'(u), this warp's columns of every 128-unit half
         if (!(ok = ewait(&bars[DG_FULL], i & 1, abort_flag))) break;
         tc_fence_after();
         for (int hf = 0; hf < nh; ++hf) {
-          uint32_t dg[2][32];
-          tmem_ld32(trow + hf * 128 + sub * 64, dg[0]);
-          tmem_ld32(trow + hf * 128 + sub * 64 + 32, dg[1]);
+          uint32_t dg[32];
+          tmem_ld32(trow + hf * 128 + sub * 32, dg);
           tmem_ld_wait();
           if (hf == nh - 1) {
             tc_fence_before();
             warp_arrive(&bars[DG_FREE], lane);
           }
-          const int c0 = hf * 128 + sub * 64;
+          const int c0 = hf * 128 + sub * 32;
           if (t < 0) continue;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 4; ++j) {
             const uint4 wp = reinterpret_cast<const uint4*>(gp_row + c0)[j];
             const __half2* hp = reinterpret_cast<const __half2*>(&wp);
-            const uint32_t* gg = &dg[j >> 2][(j & 3) * 8];
+            const uint32_t* gg = &dg[8 * j];
             float du[8];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -519,14 +526,13 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             reinterpret_cast<uint4*>((__half*)a.DUout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
           }
         }
-      } else if (!a.gather) {
-        float* es = esum + par * 256;
-        if (sub == 1) {
-          es[128 + row] = e;
+      } else if (!kGather) {  // the row's error: sub 0 adds the partial sums of subs 1-3
+        if (sub != 0) {
+          esum[(sub - 1) * 128 + row] = e;
           warp_arrive(&bars[E_READY0 + par], lane);
         } else {
           if (!(ok = ewait(&bars[E_READY0 + par], (i >> 1) & 1, abort_flag))) break;
-          if (t >= 0) a.err[(size_t)x.seg * a.T + t] = e + es[128 + row];
+          if (t >= 0) a.err[(size_t)x.seg * a.T + t] = ((e + esum[row]) + esum[128 + row]) + esum[256 + row];
         }
       }
     }
@@ -576,9 +582,10 @@ cudaError_t launch_pack_predict_tc(const PredictArgs& a, const CUtensorMap& mKt,
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(n_items < sms ? n_items : sms);
-  cudaError_t e = cudaFuncSetAttribute(pack_predict_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  auto kern = a.fit ? pack_predict_tc_kernel<2> : (a.gather ? pack_predict_tc_kernel<1> : pack_predict_tc_kernel<0>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  pack_predict_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mKt, mW1, mWl, mW2, a);
+  kern<<<grid, kThreads, kSmemBytes, st>>>(mKt, mW1, mWl, mW2, a);
   return cudaGetLastError();
 }
 
