@@ -349,7 +349,9 @@ def decode_launches_per_step(w: synth.Workload, n_sel: int) -> int:
 # in one ncu capture of the decode kernel source whose SHA-256 prefix is given. Reported as
 # roofline.traffic only while that source is unchanged; otherwise traffic is null.
 NCU_TRAFFIC = {
-    "mistral_group_32k": ("0f7b02d23a7ebf44", 76.96e6 + 0.56e6),
+    # prep + pair + combine kernels of one step
+    "llama_262k_full": ("3e3fbe5071b267e3", 2.651e6 + 567.557e6 + 0.457e6 + 2.041e6),
+    "mistral_group_32k": ("3e3fbe5071b267e3", 2.7e6 + 76.9e6 + 0.1e6 + 2.0e6),
 }
 
 
