@@ -43,7 +43,6 @@ struct PredictArgs {
   void* Rout;            // fit: [B * L * Hkv, T, 128] fp16
   void* Gout;            // fit: [B * L * Hkv, T, H] fp16
   void* DUout;           // fit: [B * L * Hkv, T, H] fp16
-  void* GP;              // fit: per-CTA scratch [grid, 128, H] fp16 (GELU' of the tile's rows)
   const void* Kt;        // [B, T, D] fp16 rebuilt keys of every (layer, KV head)
   const void* V;         // [B, L, T, Hkv, 128] bf16
   const void* b1;        // [(B,) L, Hkv, H] bf16

@@ -41,7 +41,7 @@ bool pack_tc_supported(const lr_cache_shape& s);
 // Test-time fitting: workspace layout and the whole fit (rebuilt keys, then n_steps of
 // forward, gradient and update launches).
 struct FitPlan {
-  size_t kt_off, r_off, g_off, du_off, gp_off, grad_off, w1h_off, wlh_off, w2h_off, ones_off, ws_bytes;
+  size_t kt_off, r_off, g_off, du_off, grad_off, w1h_off, wlh_off, w2h_off, ones_off, ws_bytes;
   int n_wh, gstride, grid;
 };
 FitPlan plan_fit(const lr_cache_shape& s, int per_sequence, int sm_count);

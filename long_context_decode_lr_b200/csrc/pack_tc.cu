@@ -13,9 +13,10 @@
 //   gather mode: the residual row res_val[seg, i] = round(d) of the tokens t = res_idx[seg, i]
 //                that the top-k step kept, recomputed for those rows only;
 //   fit mode:    the pieces of one gradient step of test-time fitting (explainer, paragraph on
-//                prefill cost): R = v_hat - v, g = GELU(u) and, after one more MMA
-//                MMA4 dG = R W2 (M 128, N H, K 128; W2 read MN-major from the same tile),
-//                dU' = dG * GELU'(u), all stored (fp16) for the gradient contractions.
+//                prefill cost): R = v_hat - v, g = GELU(u) and, after one more MMA per
+//                128-unit half, MMA4 dG = R W2_half (M 128, N 128, K 128; W2 read MN-major from
+//                the same tile, into TMEM columns 384-511), dU' = dG * GELU'(u) with u read
+//                again from TMEM; R, g and dU' are stored (fp16) for the gradient contractions.
 // Operands are fp16 with fp32 accumulation; GELU is the tanh form fitted to x Phi(x) (within
 // 2.71e-4). A CTA owns a contiguous range of (segment, tile) items; the segment's weights
 // (W1, W_lin, W2 as fp16, 160 KB at H = 256) stay in shared memory while its tiles stream.
@@ -284,12 +285,17 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           cur_wh = x.wh;
         }
         if (!(ok = mbar_wait(&bars[K_FULL], i & 1, abort_flag))) break;
-        // U's columns are free again once the previous tile's GELU read them (fit mode: once
-        // its dG, which reuses them, was read)
-        if (i > 0 && !(ok = mbar_wait(&bars[kFit ? DG_FREE : U_FREE], (i - 1) & 1, abort_flag))) break;
-        if (i >= 2 && !(ok = mbar_wait(&bars[V_FREE0 + (i & 1)], ((i >> 1) - 1) & 1, abort_flag))) break;
+        // U's columns are free again once the previous tile read them (the GELU branch; in
+        // fitting mode also GELU' in the last phase). v_hat is double-buffered, except in fitting
+        // mode, where columns 384-511 hold dG.
+        if (i > 0 && !(ok = mbar_wait(&bars[U_FREE], (i - 1) & 1, abort_flag))) break;
+        if (kFit) {
+          if (i > 0 && !(ok = mbar_wait(&bars[V_FREE0], (i - 1) & 1, abort_flag))) break;
+        } else {
+          if (i >= 2 && !(ok = mbar_wait(&bars[V_FREE0 + (i & 1)], ((i >> 1) - 1) & 1, abort_flag))) break;
+        }
         tc_fence_after();
-        const uint32_t vcol = tmem + 256 + 128 * (i & 1);
+        const uint32_t vcol = tmem + 256 + (kFit ? 0 : 128 * (i & 1));
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_f16_ss(tmem, sw128_desc(kt + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
@@ -312,16 +318,21 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           if (hf < nh - 1) mma_commit(&bars[G0_FREE]);
         }
         if (!ok) break;
-        mma_commit(&bars[V_FULL0 + (i & 1)]);
-        if (kFit) {  // MMA4: dG = R W2 with R in the G0 buffer, W2 read MN-major
+        mma_commit(&bars[V_FULL0 + (kFit ? 0 : (i & 1))]);
+        if (kFit) {  // MMA4, per 128-unit half: dG = R W2_half (R in G0, W2 read MN-major) -> cols 384+
           if (!(ok = mbar_wait(&bars[R_READY], i & 1, abort_flag))) break;
-          tc_fence_after();
-          const uint32_t id_dg = idesc_f16_f32(128, H, false, true);
+          const uint32_t id_dg = idesc_f16_f32(128, 128, false, true);
+          for (int hf = 0; hf < nh && ok; ++hf) {
+            const int c = i * nh + hf - 1;  // DG_FREE completion that frees the dG columns
+            if (c >= 0 && !(ok = mbar_wait(&bars[DG_FREE], c & 1, abort_flag))) break;
+            tc_fence_after();
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks)
-            mma_f16_ss(tmem, sw128_desc(g0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                       sw128_desc(w2 + ks * 2048, 16384, 1024), id_dg, ks != 0);
-          mma_commit(&bars[DG_FULL]);
+            for (int ks = 0; ks < 8; ++ks)
+              mma_f16_ss(tmem + 384, sw128_desc(g0 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                         sw128_desc(w2 + 2 * hf * 16384 + ks * 2048, 16384, 1024), id_dg, ks != 0);
+            mma_commit(&bars[DG_FULL]);
+          }
+          if (!ok) break;
         }
         mma_commit(&bars[G0_FREE]);
       }
@@ -338,7 +349,6 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     const int row = q * 32 + lane;
     const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
     float* esum = reinterpret_cast<float*>(sm + kOffEsum);
-    __half* gp_row = kFit ? (__half*)a.GP + ((size_t)blockIdx.x * 128 + row) * H : nullptr;
     bool ok = true;
     if (it0 < it1) {  // the first tile's value rows start coming from HBM into L2
       const Item x0 = item_of(a, it0, n_t);
@@ -371,7 +381,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         uint32_t u[32];
         tmem_ld32(trow + c0, u);
         tmem_ld_wait();
-        if (hf == nh - 1) {
+        if (!kFit && hf == nh - 1) {  // fitting mode reads U again for GELU'
           tc_fence_before();
           warp_arrive(&bars[U_FREE], lane);
         }
@@ -396,13 +406,9 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
               bb[2 * c + 1] = f.y;
             }
           }
-          float g[8], gp[8];
+          float g[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float xv = __uint_as_float(u[8 * j + c]) + bb[c];
-            if (kFit) gelu_and_grad(xv, g[c], gp[c]);
-            else g[c] = gelu_f32(xv);
-          }
+          for (int c = 0; c < 8; ++c) g[c] = gelu_f32(__uint_as_float(u[8 * j + c]) + bb[c]);
           uint4 w;
           w.x = pack_f16x2_sat(g[0], g[1]);
           w.y = pack_f16x2_sat(g[2], g[3]);
@@ -410,15 +416,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           w.w = pack_f16x2_sat(g[6], g[7]);
           const int q16 = 4 * (sub & 1) + j;  // 16-byte chunk of the row within the atom
           *reinterpret_cast<uint4*>(gt + ((q16 ^ (row & 7)) << 4)) = w;
-          if (kFit) {
-            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Gout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
-            uint4 wp;
-            wp.x = pack_f16x2_sat(gp[0], gp[1]);
-            wp.y = pack_f16x2_sat(gp[2], gp[3]);
-            wp.z = pack_f16x2_sat(gp[4], gp[5]);
-            wp.w = pack_f16x2_sat(gp[6], gp[7]);
-            reinterpret_cast<uint4*>(gp_row + c0)[j] = wp;
-          }
+          if (kFit && t >= 0) reinterpret_cast<uint4*>((__half*)a.Gout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
         }
         fence_proxy_async_smem();
         warp_arrive(&bars[G_READY0 + hf], lane);
@@ -432,7 +430,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
 #pragma unroll
         for (int j = 0; j < 4; ++j) vrow[j] = t >= 0 ? __ldg(vsrc + j) : make_uint4(0, 0, 0, 0);
       }
-      if (!(ok = ewait(&bars[V_FULL0 + par], (i >> 1) & 1, abort_flag))) break;
+      if (!(ok = ewait(&bars[V_FULL0 + (kFit ? 0 : par)], kFit ? (i & 1) : ((i >> 1) & 1), abort_flag))) break;
       tc_fence_after();
       float e = 0.f;
       {
@@ -442,10 +440,10 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
                                                   : nullptr;
         uint8_t* rt = sm + kOffG0 + (sub >> 1) * 16384 + row * 128;  // fit: R as the A operand of MMA4
         uint32_t vh[32];
-        tmem_ld32(trow + 256 + 128 * par + sub * 32, vh);
+        tmem_ld32(trow + 256 + (kFit ? 0 : 128 * par) + sub * 32, vh);
         tmem_ld_wait();
         tc_fence_before();
-        warp_arrive(&bars[V_FREE0 + par], lane);
+        warp_arrive(&bars[V_FREE0 + (kFit ? 0 : par)], lane);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float v[8], bb[8];
@@ -493,37 +491,45 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       if (kFit) {
         fence_proxy_async_smem();
         warp_arrive(&bars[R_READY], lane);
-        // ---- dU' = (R W2) * GELU'(u), this warp's columns of every 128-unit half
-        if (!(ok = ewait(&bars[DG_FULL], i & 1, abort_flag))) break;
-        tc_fence_after();
-        for (int hf = 0; hf < nh; ++hf) {
-          uint32_t dg[32];
-          tmem_ld32(trow + hf * 128 + sub * 32, dg);
-          tmem_ld_wait();
-          if (hf == nh - 1) {
-            tc_fence_before();
-            warp_arrive(&bars[DG_FREE], lane);
-          }
+        // ---- dU' = (R W2) * GELU'(u) per 128-unit half; u = U + b1 is read again from TMEM
+        for (int hf = 0; hf < nh && ok; ++hf) {
+          if (!(ok = ewait(&bars[DG_FULL], (i * nh + hf) & 1, abort_flag))) break;
+          tc_fence_after();
           const int c0 = hf * 128 + sub * 32;
-          if (t < 0) continue;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 wp = reinterpret_cast<const uint4*>(gp_row + c0)[j];
-            const __half2* hp = reinterpret_cast<const __half2*>(&wp);
-            const uint32_t* gg = &dg[8 * j];
-            float du[8];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const float2 f = __half22float2(hp[c]);
-              du[2 * c] = __uint_as_float(gg[2 * c]) * f.x;
-              du[2 * c + 1] = __uint_as_float(gg[2 * c + 1]) * f.y;
+          uint32_t dg[32];
+          tmem_ld32(trow + 384 + sub * 32, dg);
+          tmem_ld_wait();
+          tc_fence_before();
+          warp_arrive(&bars[DG_FREE], lane);  // the next half's dG may overwrite the columns
+          for (int ch = 0; ch < 2; ++ch) {    // U in two 16-column pieces
+            uint32_t uu[16];
+            tmem_ld16(trow + c0 + 16 * ch, uu);
+            tmem_ld_wait();
+            if (hf == nh - 1 && ch == 1) {
+              tc_fence_before();
+              warp_arrive(&bars[U_FREE], lane);
             }
-            uint4 w;
-            w.x = pack_f16x2_sat(du[0], du[1]);
-            w.y = pack_f16x2_sat(du[2], du[3]);
-            w.z = pack_f16x2_sat(du[4], du[5]);
-            w.w = pack_f16x2_sat(du[6], du[7]);
-            reinterpret_cast<uint4*>((__half*)a.DUout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
+            if (t < 0) continue;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+              const int j = 2 * ch + jj;
+              const float4 f0 = __ldg(reinterpret_cast<const float4*>(b1f + c0 + 8 * j));
+              const float4 f1 = __ldg(reinterpret_cast<const float4*>(b1f + c0 + 8 * j) + 1);
+              const float bb[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+              float du[8];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                float g, gp;
+                gelu_and_grad(__uint_as_float(uu[8 * jj + c]) + bb[c], g, gp);
+                du[c] = __uint_as_float(dg[8 * j + c]) * gp;
+              }
+              uint4 w;
+              w.x = pack_f16x2_sat(du[0], du[1]);
+              w.y = pack_f16x2_sat(du[2], du[3]);
+              w.z = pack_f16x2_sat(du[4], du[5]);
+              w.w = pack_f16x2_sat(du[6], du[7]);
+              reinterpret_cast<uint4*>((__half*)a.DUout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
+            }
           }
         }
       } else if (!kGather) {  // the row's error: sub 0 adds the partial sums of subs 1-3

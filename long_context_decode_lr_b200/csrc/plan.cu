@@ -289,8 +289,7 @@ FitPlan plan_fit(const lr_cache_shape& s, int per_sequence, int sm_count) {
   p.r_off = align256(p.kt_off + (size_t)s.batch * T * D * 2);
   p.g_off = align256(p.r_off + segs * T * 128 * 2);
   p.du_off = align256(p.g_off + segs * T * H * 2);
-  p.gp_off = align256(p.du_off + segs * T * H * 2);
-  p.grad_off = align256(p.gp_off + (size_t)sm_count * 128 * H * 2);
+  p.grad_off = align256(p.du_off + segs * T * H * 2);
   p.w1h_off = align256(p.grad_off + (size_t)p.n_wh * p.gstride * 4);
   p.wlh_off = align256(p.w1h_off + (size_t)p.n_wh * H * 128 * 2);
   p.w2h_off = align256(p.wlh_off + (size_t)p.n_wh * 128 * 128 * 2);
@@ -359,7 +358,7 @@ cudaError_t launch_fit(const lr_cache_shape& s, const FitCall& c, const FitPlan&
   p.gather = false;
   p.fit = true;
   p.Kt = Kt; p.V = c.V; p.b1 = c.b1; p.b2 = nullptr; p.b1f = c.b1; p.b2f = c.b2;
-  p.Rout = ws + plan.r_off; p.Gout = ws + plan.g_off; p.DUout = ws + plan.du_off; p.GP = ws + plan.gp_off;
+  p.Rout = ws + plan.r_off; p.Gout = ws + plan.g_off; p.DUout = ws + plan.du_off;
   p.errword = errword;
   tc::FitGradArgs ga{};
   ga.B = s.batch; ga.T = s.T; ga.L = s.n_layers; ga.Hkv = s.n_kv_heads; ga.H = s.hidden;
