@@ -40,8 +40,6 @@ struct PredictArgs {
   bool fit;
   const float* b1f;      // fit: [(B,) L, Hkv, H] fp32
   const float* b2f;      // fit: [(B,) L, Hkv, 128] fp32 or null
-  void* Rout;            // fit: [B * L * Hkv, T, 128] fp16
-  void* Gout;            // fit: [B * L * Hkv, T, H] fp16
   void* DUout;           // fit: [B * L * Hkv, T, H] fp16
   const void* Kt;        // [B, T, D] fp16 rebuilt keys of every (layer, KV head)
   const void* V;         // [B, L, T, Hkv, 128] bf16
@@ -56,8 +54,11 @@ struct PredictArgs {
 // [S * L * Hkv * H, 128], box {64, 128}; mWl over the fp16 W_lin copy [S * L * Hkv * 128, 128],
 // box {64, 128}; mW2 over the fp16 W2 copy [S * L * Hkv * 128, H], box {64, 128}
 // (S = B with per-sequence predictors, else 1).
+// Fitting mode also takes mG over g [segs, T, H] and mR over R [segs, T, 128] (fp16, box
+// {64, 128, 1}): the g halves and R leave shared memory through TMA stores (null elsewhere).
 cudaError_t launch_pack_predict_tc(const PredictArgs& a, const CUtensorMap& mKt, const CUtensorMap& mW1,
-                                   const CUtensorMap& mWl, const CUtensorMap& mW2, cudaStream_t st);
+                                   const CUtensorMap& mWl, const CUtensorMap& mW2, const CUtensorMap* mG,
+                                   const CUtensorMap* mR, cudaStream_t st);
 
 // fp16 copies of the predictor weights (saturating): W1 [n, H, 128], W_lin [n, 128, 128],
 // W2 [n, 128, H] for n = S * L * Hkv heads.

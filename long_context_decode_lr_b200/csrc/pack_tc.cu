@@ -54,7 +54,7 @@ constexpr int kSmemBytes = kOffMisc + 64;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
 enum PBar { W_FULL, W_FREE, K_FULL, K_FREE, U_FULL, U_FREE, G_READY0, G_READY1, G0_FREE, V_FULL0, V_FULL1,
-            V_FREE0, V_FREE1, E_READY0, E_READY1, DRAIN, R_READY, DG_FULL, DG_FREE, N_PBARS };
+            V_FREE0, V_FREE1, E_READY0, E_READY1, DRAIN, R_READY, DG_FULL, DG_FREE, G_STORED, N_PBARS };
 static_assert(N_PBARS * 8 <= 192, "barrier area");
 
 constexpr float kGeluC1 = 0.80015708f;  // tanh-form GELU: c1, c3 minimise the largest error
@@ -138,6 +138,7 @@ template <int kMode>  // 0 error of every token, 1 residual rows of the kept tok
 __global__ void __launch_bounds__(kThreads, 1)
 pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_constant__ CUtensorMap mapW1,
                        const __grid_constant__ CUtensorMap mapWl, const __grid_constant__ CUtensorMap mapW2,
+                       const __grid_constant__ CUtensorMap mapG, const __grid_constant__ CUtensorMap mapR,
                        const PredictArgs a) {
   constexpr bool kGather = kMode == 1, kFit = kMode == 2;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -176,6 +177,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
     mbar_init(&bars[R_READY], kEpiWarps);
     mbar_init(&bars[DG_FULL], 1);
     mbar_init(&bars[DG_FREE], kEpiWarps);
+    mbar_init(&bars[G_STORED], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -386,9 +388,14 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           warp_arrive(&bars[U_FREE], lane);
         }
         // G0's previous reader is done: the last MMA of the previous tile (commit i nh - 1), or
-        // MMA3b of half 0 of this tile (commit i nh)
+        // MMA3b of half 0 of this tile (commit i nh); in fitting mode also the TMA store of
+        // G0's previous contents (the previous tile's R, or this tile's half 0)
         const int commit = hf == 0 ? i * nh - 1 : i * nh;
         if (commit >= 0 && !(ok = ewait(&bars[G0_FREE], commit & 1, abort_flag))) break;
+        if (kFit) {
+          const int stored = i * (nh + 1) + hf - 1;
+          if (stored >= 0 && !(ok = ewait(&bars[G_STORED], stored & 1, abort_flag))) break;
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float bb[8];
@@ -416,10 +423,18 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
           w.w = pack_f16x2_sat(g[6], g[7]);
           const int q16 = 4 * (sub & 1) + j;  // 16-byte chunk of the row within the atom
           *reinterpret_cast<uint4*>(gt + ((q16 ^ (row & 7)) << 4)) = w;
-          if (kFit && t >= 0) reinterpret_cast<uint4*>((__half*)a.Gout + ((size_t)x.seg * a.T + t) * H + c0)[j] = w;
         }
         fence_proxy_async_smem();
         warp_arrive(&bars[G_READY0 + hf], lane);
+        if (kFit && warp == 2 && lane == 0) {  // the storer: g of this half to global memory
+          if (!(ok = mbar_wait(&bars[G_READY0 + hf], i & 1, abort_flag))) break;
+          for (int at = 0; at < 2; ++at)
+            tma_store_3d(&mapG, sm + kOffG0 + at * 16384, hf * 128 + 64 * at, x.tile * 128, x.seg);
+          bulk_commit_group();
+          bulk_wait_read_le0();
+          mbar_arrive(&bars[G_STORED]);
+        }
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       }
       if (!ok) break;
       // ---- value prediction done: d = v - (v_hat + b2); the value row is loaded first
@@ -439,6 +454,10 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
         __nv_bfloat16* out = (kGather && t >= 0) ? (__nv_bfloat16*)a.res_val + ((size_t)x.seg * a.k + ir) * 128 + sub * 32
                                                   : nullptr;
         uint8_t* rt = sm + kOffG0 + (sub >> 1) * 16384 + row * 128;  // fit: R as the A operand of MMA4
+        if (kFit) {  // the store of the last g half has read G0
+          const int stored = i * (nh + 1) + nh - 1;
+          if (!(ok = ewait(&bars[G_STORED], stored & 1, abort_flag))) break;
+        }
         uint32_t vh[32];
         tmem_ld32(trow + 256 + (kFit ? 0 : 128 * par) + sub * 32, vh);
         tmem_ld_wait();
@@ -484,13 +503,20 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
             w.w = pack_f16x2_sat(-d[6], -d[7]);
             const int q16 = 4 * (sub & 1) + j;
             *reinterpret_cast<uint4*>(rt + ((q16 ^ (row & 7)) << 4)) = w;
-            if (t >= 0) reinterpret_cast<uint4*>((__half*)a.Rout + ((size_t)x.seg * a.T + t) * 128 + sub * 32)[j] = w;
           }
         }
       }
       if (kFit) {
         fence_proxy_async_smem();
         warp_arrive(&bars[R_READY], lane);
+        if (warp == 2 && lane == 0) {  // the storer: R to global memory
+          if (!(ok = mbar_wait(&bars[R_READY], i & 1, abort_flag))) break;
+          for (int at = 0; at < 2; ++at) tma_store_3d(&mapR, sm + kOffG0 + at * 16384, 64 * at, x.tile * 128, x.seg);
+          bulk_commit_group();
+          bulk_wait_read_le0();
+          mbar_arrive(&bars[G_STORED]);
+        }
+        if (!__all_sync(0xffffffffu, ok)) break;
         // ---- dU' = (R W2) * GELU'(u) per 128-unit half; u = U + b1 is read again from TMEM
         for (int hf = 0; hf < nh && ok; ++hf) {
           if (!(ok = ewait(&bars[DG_FULL], (i * nh + hf) & 1, abort_flag))) break;
@@ -546,6 +572,7 @@ pack_predict_tc_kernel(const __grid_constant__ CUtensorMap mapKt, const __grid_c
       *abort_flag = 1;
       flag_error(a.errword, LR_DEVERR_TIMEOUT);
     }
+    if (kFit && warp == 2 && lane == 0) bulk_wait_all();  // the stored g and R rows have landed
   }
   __syncwarp();
   tc_fence_before();
@@ -581,7 +608,8 @@ __global__ void weights_f16_kernel(const __nv_bfloat16* __restrict__ W1, const _
 }  // namespace
 
 cudaError_t launch_pack_predict_tc(const PredictArgs& a, const CUtensorMap& mKt, const CUtensorMap& mW1,
-                                   const CUtensorMap& mWl, const CUtensorMap& mW2, cudaStream_t st) {
+                                   const CUtensorMap& mWl, const CUtensorMap& mW2, const CUtensorMap* mG,
+                                   const CUtensorMap* mR, cudaStream_t st) {
   const int n_t = a.gather ? (a.k + 127) / 128 : (a.T + 127) / 128;
   const long long n_items = (long long)a.B * a.L * a.Hkv * n_t;
   if (n_items == 0) return cudaSuccess;
@@ -591,7 +619,8 @@ cudaError_t launch_pack_predict_tc(const PredictArgs& a, const CUtensorMap& mKt,
   auto kern = a.fit ? pack_predict_tc_kernel<2> : (a.gather ? pack_predict_tc_kernel<1> : pack_predict_tc_kernel<0>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(mKt, mW1, mWl, mW2, a);
+  // the g and R maps are used in fitting mode only; the other modes get placeholders
+  kern<<<grid, kThreads, kSmemBytes, st>>>(mKt, mW1, mWl, mW2, mG ? *mG : mKt, mR ? *mR : mKt, a);
   return cudaGetLastError();
 }
 

@@ -263,14 +263,14 @@ cudaError_t launch_pack_tc(const PackArgs& a, const PackPlan& plan, cudaStream_t
   p.Kt = Kt; p.V = a.V; p.b1 = a.b1; p.b2 = a.b2; p.err = a.err;
   p.res_idx = a.res_idx; p.res_val = a.res_val; p.errword = a.errword;
   // P3 + P4: predictor and per-token error of every token
-  if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+  if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, nullptr, nullptr, st)) != cudaSuccess) return e;
   // P5: exact top-k per (sequence, layer, KV head)
   const int n_seg = a.B * a.L * a.Hkv;
   if ((e = launch_topk(a.err, n_seg, a.T, a.k, a.res_idx, st)) != cudaSuccess) return e;
   // P6: residual rows of the kept tokens, recomputed; block pointers
   if (a.k > 0) {
     p.gather = true;
-    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, nullptr, nullptr, st)) != cudaSuccess) return e;
   }
   if (a.res_ptr) return launch_block_ptr(a.res_idx, n_seg, a.k, a.T, a.res_ptr, st);
   return cudaSuccess;
@@ -358,7 +358,15 @@ cudaError_t launch_fit(const lr_cache_shape& s, const FitCall& c, const FitPlan&
   p.gather = false;
   p.fit = true;
   p.Kt = Kt; p.V = c.V; p.b1 = c.b1; p.b2 = nullptr; p.b1f = c.b1; p.b2f = c.b2;
-  p.Rout = ws + plan.r_off; p.Gout = ws + plan.g_off; p.DUout = ws + plan.du_off;
+  p.DUout = ws + plan.du_off;
+  CUtensorMap mGst, mRst;  // g and R leave the forward kernel through TMA stores
+  {
+    const cuuint64_t dR[3] = {128, T, segs}, sR[2] = {256, T * 256};
+    const cuuint64_t dU[3] = {H, T, segs}, sU[2] = {H * 2, T * H * 2};
+    const cuuint32_t b128[3] = {64, 128, 1};
+    if (!tile_map(&mGst, F16, ws + plan.g_off, 3, dU, sU, b128) || !tile_map(&mRst, F16, ws + plan.r_off, 3, dR, sR, b128))
+      return cudaErrorInvalidValue;
+  }
   p.errword = errword;
   tc::FitGradArgs ga{};
   ga.B = s.batch; ga.T = s.T; ga.L = s.n_layers; ga.Hkv = s.n_kv_heads; ga.H = s.hidden;
@@ -375,7 +383,7 @@ cudaError_t launch_fit(const lr_cache_shape& s, const FitCall& c, const FitPlan&
   u.lr = c.lr;
   u.scale = 2.0f / ((float)s.T * (c.per_sequence ? 1.0f : (float)s.batch) * (float)s.head_dim);
   for (int step = 0; step < c.n_steps; ++step) {
-    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, st)) != cudaSuccess) return e;
+    if ((e = tc::launch_pack_predict_tc(p, mKt, mW1, mWl, mW2, &mGst, &mRst, st)) != cudaSuccess) return e;
     if ((e = tc::launch_fit_grad(ga, mR, mDU, mG, mKt64, mOnes, st)) != cudaSuccess) return e;
     if (step == c.n_steps - 1) {
       u.out_Wl = c.out_Wl; u.out_W1 = c.out_W1; u.out_b1 = c.out_b1; u.out_W2 = c.out_W2; u.out_b2 = c.out_b2;

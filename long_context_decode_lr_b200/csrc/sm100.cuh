@@ -133,6 +133,8 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until at most one committed bulk group still reads shared memory.
 __device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// Waits until no committed bulk group still reads shared memory.
+__device__ __forceinline__ void bulk_wait_read_le0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Waits until every committed bulk group has completed (its global writes included).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
