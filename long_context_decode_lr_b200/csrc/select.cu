@@ -117,15 +117,16 @@ __global__ void __launch_bounds__(SEL_THREADS) select_qhat_kernel(SelectArgs a) 
 constexpr int kScBlocks = 32;  // blocks per CTA (4 per warp)
 constexpr int kScPairs = 32;   // (KV head, query head) pairs per pass: one per lane
 constexpr int kScCols = 128;   // rank columns staged per pass
+constexpr int kScPad = 4;      // Qhat row padding: 16-byte rows without bank conflicts
 static_assert(kScBlocks == kScPairs && kScBlocks == 4 * SEL_THREADS / 32, "staging loop and warp split");
 
 // Scores [B, Hkv, nblk]: one CTA per 32 blocks of a sequence. Lane l of every warp owns the
 // (KV head, query head) pair l of the current pass and accumulates its dot products with the
-// warp's 4 block means; rank columns are staged 128 at a time (Qhat rows padded against bank
-// conflicts, block means read as broadcasts).
+// warp's 4 block means; rank columns are staged 128 at a time and read four at a time (Qhat
+// rows padded against bank conflicts, block means read as broadcasts).
 __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a) {
-  __shared__ float qs[kScPairs][kScCols + 1];
-  __shared__ float as[kScBlocks][kScCols];
+  __shared__ __align__(16) float qs[kScPairs][kScCols + kScPad];
+  __shared__ __align__(16) float as[kScBlocks][kScCols];
   __shared__ float dots[kScBlocks][kScPairs + 1];
   const int j0 = blockIdx.x * kScBlocks, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -138,19 +139,30 @@ __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a)
     const int np = min(pass, P - p0);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int c0 = 0; c0 < r; c0 += kScCols) {
-      const int nc = min(kScCols, r - c0);
+      const int nc = min(kScCols, r - c0);  // r is a multiple of 8, so nc is a multiple of 4
       __syncthreads();
-      for (int i = tid; i < kScPairs * kScCols; i += SEL_THREADS) {
-        const int p = i / kScCols, c = i % kScCols;
-        qs[p][c] = (p < np && c < nc) ? qh[(size_t)(p0 + p) * r + c0 + c] : 0.f;
-        as[p][c] = (p < nb && c < nc) ? ab[(size_t)p * r + c0 + c] : 0.f;
+      for (int i = tid; i < kScPairs * (kScCols / 4); i += SEL_THREADS) {
+        const int p = i / (kScCols / 4), c = 4 * (i % (kScCols / 4));
+        const bool cin = c < nc;
+        *reinterpret_cast<float4*>(&qs[p][c]) =
+            (p < np && cin) ? __ldg(reinterpret_cast<const float4*>(qh + (size_t)(p0 + p) * r + c0 + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4*>(&as[p][c]) =
+            (p < nb && cin) ? __ldg(reinterpret_cast<const float4*>(ab + (size_t)p * r + c0 + c))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       __syncthreads();
 #pragma unroll 4
-      for (int c = 0; c < kScCols; ++c) {
-        const float qv = qs[lane][c];
+      for (int c = 0; c < kScCols; c += 4) {
+        const float4 qv = *reinterpret_cast<const float4*>(&qs[lane][c]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = fmaf(qv, as[warp * 4 + i][c], acc[i]);
+        for (int i = 0; i < 4; ++i) {
+          const float4 av = *reinterpret_cast<const float4*>(&as[warp * 4 + i][c]);
+          acc[i] = fmaf(qv.x, av.x, acc[i]);
+          acc[i] = fmaf(qv.y, av.y, acc[i]);
+          acc[i] = fmaf(qv.z, av.z, acc[i]);
+          acc[i] = fmaf(qv.w, av.w, acc[i]);
+        }
       }
     }
     __syncthreads();

@@ -285,7 +285,7 @@ __global__ void block_ptr_kernel(const int* __restrict__ idx, int n_seg, int k, 
 
 cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out, cudaStream_t st) {
   if (n_seg == 0 || k == 0) return cudaSuccess;
-  if (T >= 16384 && k < T) {  // long segments: one cluster of CTAs per segment
+  if (T >= 4096 && k < T) {  // long segments: one cluster of CTAs per segment
     topk_cluster_kernel<<<dim3(kTkCluster, n_seg), TKC_THREADS, 0, st>>>(err, T, k, idx_out);
     return cudaGetLastError();
   }
