@@ -260,7 +260,8 @@ size_t lr_select_workspace_bytes(const lr_cache_shape* s, int32_t n_q_heads) {
   const size_t nblk = (size_t)lr::ceil_div(s->T, LR_BLOCK_TOKENS);
   const size_t qhat = (size_t)s->batch * n_q_heads * s->rank * sizeof(float);
   const size_t scores = (size_t)s->batch * s->n_kv_heads * nblk * sizeof(float);
-  return 256 + ((qhat + 255) & ~(size_t)255) + ((scores + 255) & ~(size_t)255);
+  const size_t partial = (size_t)lr::select_rank_splits(s->rank) * s->batch * nblk * n_q_heads * sizeof(float);
+  return 256 + ((qhat + 255) & ~(size_t)255) + ((scores + 255) & ~(size_t)255) + ((partial + 255) & ~(size_t)255);
 }
 
 lr_status lr_block_means(const lr_cache_shape* s, const void* A, float* Abar, lr_stream_t stream) {
@@ -299,7 +300,10 @@ lr_status lr_select_blocks(const lr_cache_shape* s, int32_t layer, int32_t n_q_h
   a.q = q; a.abar = Abar; a.Bt = Bt;
   const size_t qhat = (size_t)s->batch * n_q_heads * s->rank * sizeof(float);
   a.qhat = (float*)((char*)ws + 256);
+  const size_t scores_bytes = (size_t)s->batch * s->n_kv_heads * nblk * sizeof(float);
   a.scores = scores_out ? scores_out : (float*)((char*)ws + 256 + ((qhat + 255) & ~(size_t)255));
+  a.partial = (float*)((char*)ws + 256 + ((qhat + 255) & ~(size_t)255) + ((scores_bytes + 255) & ~(size_t)255));
+  a.n_split = lr::select_rank_splits(s->rank);
   a.blocks_out = block_list;
   const cudaError_t e = lr::launch_select_blocks(a, s->dtype, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "block selection launch");

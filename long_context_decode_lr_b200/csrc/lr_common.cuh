@@ -112,6 +112,8 @@ struct SelectArgs {
   const void* Bt;      // [B, D, r]
   float* qhat;         // workspace [B, Hkv, G, r]: scale * B_l^h q per query head
   float* scores;       // [B, Hkv, nblk]: the caller's scores_out, or workspace
+  float* partial;      // workspace [n_split, B, nblk, Hkv * G]: partial dot products
+  int n_split;         // rank splits of the score kernel (select_rank_splits(r))
   int* blocks_out;     // [B, Hkv, n_sel]
 };
 

@@ -34,6 +34,7 @@ cudaError_t launch_block_ptr(const int* idx, int n_seg, int k, int T, int* ptr_o
 // Block selection: block means of A (once per packed cache), mean-key block scores and
 // their top-n_sel per (sequence, KV head).
 cudaError_t launch_block_means(const void* A, int B, int T, int r, lr_dtype dt, float* abar, cudaStream_t st);
+int select_rank_splits(int r);
 cudaError_t launch_select_blocks(const SelectArgs& a, lr_dtype dt, cudaStream_t st);
 
 }  // namespace lr

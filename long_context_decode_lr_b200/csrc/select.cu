@@ -8,6 +8,10 @@
 // once per packed cache (block_means_kernel), so a selection step reads 1/64 of A. The n_sel
 // blocks of highest score per (sequence, KV head) are then chosen by the exact top-k of
 // topk.cu (ties to the lower block id, ascending).
+#include <math_constants.h>
+
+#include <algorithm>
+
 #include "lr_common.cuh"
 #include "lr_launch.h"
 
@@ -80,28 +84,39 @@ __global__ void __launch_bounds__(SEL_THREADS) block_means_kernel(const T* __res
   }
 }
 
-// Qhat [B, Hkv * G, r] fp32: one CTA per (64 rank columns, KV head, sequence). Thread
-// (dg, c) sums every fourth key dim for rank column c; a 4-way reduction in shared memory.
+// Qhat [B, Hkv * G, r] fp32: one CTA per (32 rank columns, KV head, sequence). Warp w sums
+// the key dims d = w, w + 8, ... for rank column lane (loads issued 16 at a time); an 8-way
+// reduction in shared memory.
 template <typename T>
 __global__ void __launch_bounds__(SEL_THREADS) select_qhat_kernel(SelectArgs a) {
   __shared__ float qs[8][256];
-  __shared__ float part[4][64][9];
+  __shared__ float part[8][32][9];
   const int jc = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
   const int G = a.G, hd = a.hd, r = a.r;
   const T* q = (const T*)a.q + ((size_t)b * a.Hkv + h) * G * hd;
   for (int i = tid; i < G * hd; i += SEL_THREADS) qs[i / hd][i % hd] = to_f32(q[i]) * a.scale;
   __syncthreads();
-  const int c = tid & 63, dg = tid >> 6;
-  const int j = jc * 64 + c;
+  const int c = tid & 31, dg = tid >> 5;
+  const int j = jc * 32 + c;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (j < r) {
     const size_t D = (size_t)a.L * a.Hkv * hd;
     const T* bt = (const T*)a.Bt + (size_t)b * D * r + (size_t)(a.layer * a.Hkv + h) * hd * r + j;
-    for (int d = dg; d < hd; d += 4) {
-      const float v = to_f32(bt[(size_t)d * r]);
+    for (int d0 = dg; d0 < hd; d0 += 8 * 16) {
+      float v[16];
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
-        if (g < G) acc[g] = fmaf(v, qs[g][d], acc[g]);
+      for (int u = 0; u < 16; ++u) {
+        const int d = d0 + 8 * u;
+        v[u] = d < hd ? to_f32(bt[(size_t)d * r]) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int d = d0 + 8 * u;
+        if (d >= hd) break;
+#pragma unroll
+        for (int g = 0; g < 8; ++g)
+          if (g < G) acc[g] = fmaf(v[u], qs[g][d], acc[g]);
+      }
     }
   }
 #pragma unroll
@@ -110,8 +125,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_qhat_kernel(SelectArgs a) 
   if (dg != 0 || j >= r) return;
   float* out = a.qhat + ((size_t)b * a.Hkv + h) * G * r + j;
 #pragma unroll
-  for (int g = 0; g < 8; ++g)
-    if (g < G) out[(size_t)g * r] = (part[0][c][g] + part[1][c][g]) + (part[2][c][g] + part[3][c][g]);
+  for (int g = 0; g < 8; ++g) {
+    if (g >= G) continue;
+    float x = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) x += part[w][c][g];
+    out[(size_t)g * r] = x;
+  }
 }
 
 constexpr int kScBlocks = 32;  // blocks per CTA (4 per warp)
@@ -120,14 +140,15 @@ constexpr int kScCols = 128;   // rank columns staged per pass
 constexpr int kScPad = 4;      // Qhat row padding: 16-byte rows without bank conflicts
 static_assert(kScBlocks == kScPairs && kScBlocks == 4 * SEL_THREADS / 32, "staging loop and warp split");
 
-// Scores [B, Hkv, nblk]: one CTA per 32 blocks of a sequence. Lane l of every warp owns the
-// (KV head, query head) pair l of the current pass and accumulates its dot products with the
-// warp's 4 block means; rank columns are staged 128 at a time and read four at a time (Qhat
-// rows padded against bank conflicts, block means read as broadcasts).
+// Partial dot products [n_split, B, nblk, Hkv * G]: one CTA per (32 blocks, sequence, rank
+// split); split z covers the 128-column chunks [z * n_chunks / n_split, (z + 1) * n_chunks /
+// n_split). Lane l of every warp owns the (KV head, query head) pair l of the current pass
+// and accumulates its dot products with the warp's 4 block means; rank columns are staged
+// 128 at a time and read four at a time (Qhat rows padded against bank conflicts, block
+// means read as broadcasts).
 __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a) {
   __shared__ __align__(16) float qs[kScPairs][kScCols + kScPad];
   __shared__ __align__(16) float as[kScBlocks][kScCols];
-  __shared__ float dots[kScBlocks][kScPairs + 1];
   const int j0 = blockIdx.x * kScBlocks, b = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = a.r, G = a.G, P = a.Hkv * G;
@@ -135,10 +156,13 @@ __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a)
   const float* qh = a.qhat + (size_t)b * P * r;
   const float* ab = a.abar + ((size_t)b * a.nblk + j0) * r;
   const int pass = (kScPairs / G) * G;  // whole heads per pass: a head never straddles two
+  const int n_chunks = (r + kScCols - 1) / kScCols, z = blockIdx.z;
+  const int c_begin = (z * n_chunks / a.n_split) * kScCols;
+  const int c_end = min(r, ((z + 1) * n_chunks / a.n_split) * kScCols);
   for (int p0 = 0; p0 < P; p0 += pass) {
     const int np = min(pass, P - p0);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c0 = 0; c0 < r; c0 += kScCols) {
+    for (int c0 = c_begin; c0 < c_end; c0 += kScCols) {
       const int nc = min(kScCols, r - c0);  // r is a multiple of 8, so nc is a multiple of 4
       __syncthreads();
       for (int i = tid; i < kScPairs * (kScCols / 4); i += SEL_THREADS) {
@@ -165,33 +189,48 @@ __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a)
         }
       }
     }
-    __syncthreads();
+    float* part = a.partial + (((size_t)z * a.B + b) * a.nblk + j0) * P + p0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dots[warp * 4 + i][lane] = acc[i];
-    __syncthreads();
-    // per (block, head of this pass): the largest dot product over the head's query heads
-    const int nh = np / G;
-    for (int x = tid; x < kScBlocks * kScPairs; x += SEL_THREADS) {
-      const int blk = x / kScPairs, hl = x % kScPairs;
-      if (blk >= nb || hl >= nh) continue;
-      float m = dots[blk][hl * G];
-      for (int g = 1; g < G; ++g) m = fmaxf(m, dots[blk][hl * G + g]);
-      a.scores[((size_t)b * a.Hkv + p0 / G + hl) * a.nblk + j0 + blk] = m;
+    for (int i = 0; i < 4; ++i) {
+      const int blk = warp * 4 + i;
+      if (blk < nb && lane < np) part[(size_t)blk * P + lane] = acc[i];
     }
   }
 }
 
+// Scores [B, Hkv, nblk]: s = max over the head's query heads of the summed partial dot
+// products (splits added in a fixed order).
+__global__ void __launch_bounds__(SEL_THREADS) select_reduce_kernel(SelectArgs a) {
+  const long long x = (long long)blockIdx.x * SEL_THREADS + threadIdx.x;
+  const long long n = (long long)a.B * a.Hkv * a.nblk;
+  if (x >= n) return;
+  const int j = (int)(x % a.nblk), h = (int)((x / a.nblk) % a.Hkv), b = (int)(x / ((long long)a.nblk * a.Hkv));
+  const int G = a.G, P = a.Hkv * G;
+  float m = -CUDART_INF_F;
+  for (int g = 0; g < G; ++g) {
+    float v = 0.f;
+    for (int z = 0; z < a.n_split; ++z) v += a.partial[(((size_t)z * a.B + b) * a.nblk + j) * P + h * G + g];
+    m = g == 0 ? v : fmaxf(m, v);
+  }
+  a.scores[((size_t)b * a.Hkv + h) * a.nblk + j] = m;
+}
+
 template <typename T>
 cudaError_t launch_select_t(const SelectArgs& a, cudaStream_t st) {
-  select_qhat_kernel<T><<<dim3((a.r + 63) / 64, a.Hkv, a.B), SEL_THREADS, 0, st>>>(a);
+  select_qhat_kernel<T><<<dim3((a.r + 31) / 32, a.Hkv, a.B), SEL_THREADS, 0, st>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  select_score_kernel<<<dim3((a.nblk + kScBlocks - 1) / kScBlocks, a.B), SEL_THREADS, 0, st>>>(a);
+  select_score_kernel<<<dim3((a.nblk + kScBlocks - 1) / kScBlocks, a.B, a.n_split), SEL_THREADS, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long n = (long long)a.B * a.Hkv * a.nblk;
+  select_reduce_kernel<<<(unsigned)((n + SEL_THREADS - 1) / SEL_THREADS), SEL_THREADS, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_topk(a.scores, a.B * a.Hkv, a.nblk, a.n_sel, a.blocks_out, st);
 }
 
 }  // namespace
+
+int select_rank_splits(int r) { return std::max(1, std::min(4, (r + kScCols - 1) / kScCols)); }
 
 cudaError_t launch_select_blocks(const SelectArgs& a, lr_dtype dt, cudaStream_t st) {
   if (a.B == 0 || a.nblk == 0) return cudaSuccess;

@@ -45,6 +45,47 @@ __device__ __forceinline__ int block_exclusive_scan(bool flag, int* warp_tot, in
   return before + in_warp;
 }
 
+// Digit of the kr-th largest key among those matching the current prefix, from the 256-bin
+// histogram h of the pass: the largest d with (sum of h above d) + h[d] >= kr (0 if none), and
+// kr minus the count above d. Run by one whole warp: lane l owns bins 8l .. 8l+7, a suffix
+// scan over lanes finds the lane that holds the digit, that lane scans its bins.
+__device__ __forceinline__ void find_digit_warp(const int* h, int kr, int* out_digit, int* out_kr) {
+  const int lane = threadIdx.x & 31;
+  int v[8], s = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = h[8 * lane + i];
+    s += v[i];
+  }
+  int incl = s;  // sum over lanes >= this one (higher digits)
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_down_sync(0xffffffffu, incl, o);
+    if (lane + o < 32) incl += x;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= kr);
+  if (hit == 0u) {  // fewer than kr keys left: the scan of the serial form ends at digit 0
+    const int above0 = __shfl_sync(0xffffffffu, incl, 0) - __shfl_sync(0xffffffffu, v[0], 0);
+    if (lane == 0) {
+      *out_digit = 0;
+      *out_kr = kr - above0;
+    }
+    return;
+  }
+  const int L = 31 - __clz((int)hit);
+  if (lane == L) {
+    int cum = incl - s;  // keys in the bins above this lane's
+    int d = 8 * lane + 7;
+#pragma unroll
+    for (int i = 7; i > 0; --i, --d) {
+      if (cum + v[i] >= kr) break;
+      cum += v[i];
+    }
+    *out_digit = d;
+    *out_kr = kr - cum;
+  }
+}
+
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ err, int T, int k,
                                                          int* __restrict__ out_all) {
   __shared__ int whist[TK_WARPS][256];
@@ -87,15 +128,7 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
       hist[tid] = s;
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, d = 255;
-      for (; d > 0; --d) {
-        if (cum + hist[d] >= kr) break;
-        cum += hist[d];
-      }
-      sh_digit = d;
-      sh_kr = kr - cum;
-    }
+    if (warp == 0) find_digit_warp(hist, kr, &sh_digit, &sh_kr);
     __syncthreads();
     prefix |= (uint32_t)sh_digit << shift;
     mask |= 255u << shift;
@@ -198,15 +231,7 @@ __global__ void __cluster_dims__(kTkCluster, 1, 1) __launch_bounds__(TKC_THREADS
       whist[0][tid] = s;  // the cluster's histogram
     }
     __syncthreads();
-    if (tid == 0) {
-      int cum = 0, d = 255;
-      for (; d > 0; --d) {
-        if (cum + whist[0][d] >= kr) break;
-        cum += whist[0][d];
-      }
-      sh_digit = d;
-      sh_kr = kr - cum;
-    }
+    if (warp == 0) find_digit_warp(&whist[0][0], kr, &sh_digit, &sh_kr);
     sm100::cluster_sync();  // no CTA rewrites its histogram while another still reads it
     prefix |= (uint32_t)sh_digit << shift;
     mask |= 255u << shift;
