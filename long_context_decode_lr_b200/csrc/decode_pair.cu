@@ -862,25 +862,67 @@ __global__ void __launch_bounds__(256) decode_pair_prep_kernel(PairArgs a, int n
     }
     return;
   }
-  if (tid != 0) return;
+  // One CTA per (sequence, KV head). An entry is taken when it lies in range, is above its
+  // predecessor in the list and above every taken entry before it; the largest taken entry
+  // before position k equals the largest in-range, in-order entry before k, so both the
+  // test and the output positions are prefix scans (max and count) over the list.
+  __shared__ int w_max[8], w_cnt[8];
+  __shared__ int s_bits;
   const int q = bid - n_w1 - n_q;
   const int h = q % a.Hkv, b = q / a.Hkv;
   const int* l = blocks + ((size_t)b * a.Hkv + h) * n_sel;
   int* out = a.sched + ((size_t)b * a.Hkv + h) * a.sched_stride;
-  int n = 0, prev = -1, bits = 0;
-  for (int k = 0; k < n_sel; ++k) {
-    const int v = l[k];
-    const bool bad_range = v < 0 || v >= a.nblk;
-    const bool bad_order = k > 0 && l[k - 1] >= v;
-    if (bad_range) bits |= LR_DEVERR_BLOCK_RANGE;
-    if (bad_order) bits |= LR_DEVERR_BLOCK_ORDER;
-    if (!bad_range && !bad_order && v > prev) {
-      out[1 + n++] = v;
-      prev = v;
+  const int lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_bits = 0;
+  __syncthreads();
+  int carry_max = -1, carry_n = 0, bits = 0;
+  for (int k0 = 0; k0 < n_sel; k0 += 256) {
+    const int k = k0 + tid;
+    int v = -1;
+    bool elig = false;
+    if (k < n_sel) {
+      v = l[k];
+      const bool bad_range = v < 0 || v >= a.nblk;
+      const bool bad_order = k > 0 && l[k - 1] >= v;
+      if (bad_range) bits |= LR_DEVERR_BLOCK_RANGE;
+      if (bad_order) bits |= LR_DEVERR_BLOCK_ORDER;
+      elig = !bad_range && !bad_order;
     }
+    // inclusive prefix max of eligible values within the warp, then across warps
+    int mx = elig ? v : -1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, mx, o);
+      if (lane >= o) mx = max(mx, y);
+    }
+    if (lane == 31) w_max[warp] = mx;
+    __syncthreads();
+    int before_max = carry_max;  // largest eligible value before this entry
+    for (int w = 0; w < warp; ++w) before_max = max(before_max, w_max[w]);
+    const int prev_lane = __shfl_up_sync(0xffffffffu, mx, 1);
+    if (lane > 0) before_max = max(before_max, prev_lane);
+    const bool take = elig && v > before_max;
+    // exclusive prefix count of taken entries
+    const unsigned bal = __ballot_sync(0xffffffffu, take);
+    if (lane == 0) w_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int pos = carry_n + __popc(bal & ((1u << lane) - 1u)), chunk_n = 0, chunk_max = carry_max;
+    for (int w = 0; w < 8; ++w) {
+      if (w < warp) pos += w_cnt[w];
+      chunk_n += w_cnt[w];
+      chunk_max = max(chunk_max, w_max[w]);
+    }
+    if (take) out[1 + pos] = v;
+    carry_n += chunk_n;
+    carry_max = chunk_max;
+    __syncthreads();  // w_max / w_cnt are rewritten by the next chunk
   }
-  out[0] = n;
-  if (bits) flag_error(a.err, bits);
+  if (bits) atomicOr(&s_bits, bits);
+  __syncthreads();
+  if (tid == 0) {
+    out[0] = carry_n;
+    if (s_bits) flag_error(a.err, s_bits);
+  }
 }
 
 template <int MG, bool Q2>

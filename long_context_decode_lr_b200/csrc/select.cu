@@ -201,10 +201,12 @@ __global__ void __launch_bounds__(SEL_THREADS) select_score_kernel(SelectArgs a)
 // Scores [B, Hkv, nblk]: s = max over the head's query heads of the summed partial dot
 // products (splits added in a fixed order).
 __global__ void __launch_bounds__(SEL_THREADS) select_reduce_kernel(SelectArgs a) {
+  // one thread per (sequence, block, KV head), the head fastest: a warp reads contiguous
+  // partial sums
   const long long x = (long long)blockIdx.x * SEL_THREADS + threadIdx.x;
   const long long n = (long long)a.B * a.Hkv * a.nblk;
   if (x >= n) return;
-  const int j = (int)(x % a.nblk), h = (int)((x / a.nblk) % a.Hkv), b = (int)(x / ((long long)a.nblk * a.Hkv));
+  const int h = (int)(x % a.Hkv), j = (int)((x / a.Hkv) % a.nblk), b = (int)(x / ((long long)a.nblk * a.Hkv));
   const int G = a.G, P = a.Hkv * G;
   float m = -CUDART_INF_F;
   for (int g = 0; g < G; ++g) {

@@ -86,6 +86,10 @@ __device__ __forceinline__ void find_digit_warp(const int* h, int kr, int* out_d
   }
 }
 
+// Segments of up to kTkKeys * TK_THREADS tokens: thread tid keeps the keys of tokens
+// tid + i * TK_THREADS (i < kTkKeys) in registers for all passes.
+constexpr int kTkKeys = 8;
+
 __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restrict__ err, int T, int k,
                                                          int* __restrict__ out_all) {
   __shared__ int whist[TK_WARPS][256];
@@ -100,21 +104,25 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
     for (int t = tid; t < T; t += TK_THREADS) out[t] = t;
     return;
   }
+  const int n_it = (T + TK_THREADS - 1) / TK_THREADS;  // <= kTkKeys (checked by the launcher)
+  uint32_t key[kTkKeys];
+#pragma unroll
+  for (int i = 0; i < kTkKeys; ++i) {
+    const int t = tid + i * TK_THREADS;
+    key[i] = (i < n_it && t < T) ? order_key(e[t]) : 0u;
+  }
   uint32_t prefix = 0, mask = 0;
   int kr = k;  // rank still to locate among keys that match the prefix
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int i = tid; i < TK_WARPS * 256; i += TK_THREADS) (&whist[0][0])[i] = 0;
     __syncthreads();
-    for (int t0 = 0; t0 < T; t0 += TK_THREADS) {
-      const int t = t0 + tid;
-      bool act = false;
-      int digit = 0;
-      if (t < T) {
-        const uint32_t key = order_key(e[t]);
-        act = (key & mask) == prefix;
-        digit = (key >> shift) & 255;
-      }
+#pragma unroll
+    for (int i = 0; i < kTkKeys; ++i) {
+      if (i >= n_it) break;
+      const int t = tid + i * TK_THREADS;
+      const bool act = t < T && (key[i] & mask) == prefix;
+      const int digit = (key[i] >> shift) & 255;
       const unsigned actmask = __ballot_sync(0xffffffffu, act);
       if (act) {
         const unsigned same = __match_any_sync(actmask, digit);
@@ -139,21 +147,20 @@ __global__ void __launch_bounds__(TK_THREADS) topk_kernel(const float* __restric
   const uint32_t kstar = prefix;
   const int n_tie = kr;
   int ties_before = 0, taken_before = 0;
-  for (int t0 = 0; t0 < T; t0 += TK_THREADS) {
-    const int t = t0 + tid;
-    uint32_t key = 0;
+#pragma unroll
+  for (int i = 0; i < kTkKeys; ++i) {
+    if (i >= n_it || taken_before >= k) break;
+    const int t = tid + i * TK_THREADS;
     const bool valid = t < T;
-    if (valid) key = order_key(e[t]);
-    const bool is_eq = valid && key == kstar;
+    const bool is_eq = valid && key[i] == kstar;
     int eq_total;
     const int eq_rank = ties_before + block_exclusive_scan(is_eq, warp_tot, eq_total);
-    const bool take = valid && (key > kstar || (is_eq && eq_rank < n_tie));
+    const bool take = valid && (key[i] > kstar || (is_eq && eq_rank < n_tie));
     int take_total;
     const int pos = taken_before + block_exclusive_scan(take, warp_tot, take_total);
     if (take) out[pos] = t;
     ties_before += eq_total;
     taken_before += take_total;
-    if (taken_before >= k) break;
   }
 }
 
@@ -291,6 +298,11 @@ __global__ void __cluster_dims__(kTkCluster, 1, 1) __launch_bounds__(TKC_THREADS
   }
 }
 
+__global__ void __launch_bounds__(TK_THREADS) topk_all_kernel(int T, int* __restrict__ out_all) {
+  int* out = out_all + (size_t)blockIdx.x * T;
+  for (int t = threadIdx.x; t < T; t += TK_THREADS) out[t] = t;
+}
+
 __global__ void block_ptr_kernel(const int* __restrict__ idx, int n_seg, int k, int T, int nblk,
                                  int* __restrict__ ptr) {
   const long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -312,6 +324,10 @@ cudaError_t launch_topk(const float* err, int n_seg, int T, int k, int* idx_out,
   if (n_seg == 0 || k == 0) return cudaSuccess;
   if (T >= 4096 && k < T) {  // long segments: one cluster of CTAs per segment
     topk_cluster_kernel<<<dim3(kTkCluster, n_seg), TKC_THREADS, 0, st>>>(err, T, k, idx_out);
+    return cudaGetLastError();
+  }
+  if (T > kTkKeys * TK_THREADS) {  // k == T on a long segment: every index, in order
+    topk_all_kernel<<<n_seg, TK_THREADS, 0, st>>>(T, idx_out);
     return cudaGetLastError();
   }
   topk_kernel<<<n_seg, TK_THREADS, 0, st>>>(err, T, k, idx_out);

@@ -109,6 +109,43 @@ def test_bad_block_lists_set_the_error_word():
     H.assert_attention_close(got, ref)
 
 
+def _accepted(lst, nblk):
+    """The entries a decode step keeps from a caller's block list: in range, above the entry
+    before it in the list and above every entry kept so far (the documented skipping rule)."""
+    kept, prev = [], -1
+    for k, v in enumerate(lst):
+        if v < 0 or v >= nblk or (k > 0 and lst[k - 1] >= v):
+            continue
+        if v > prev:
+            kept.append(int(v))
+            prev = v
+    return kept
+
+
+def test_long_disordered_block_lists():
+    # lists of 600 entries (three 256-entry chunks of the device-side scan), with swapped
+    # pairs, repeated entries and out-of-range values spread over the whole list
+    w = H.small(T=48000, res_pct=5)
+    p = H.packed_problem(w, sel=600)
+    q_st, q_ref = H.queries(p, 0)
+    rng = np.random.default_rng(7)
+    bad = p.blocks.copy()
+    for h in range(w.n_kv_heads):
+        for _ in range(12):
+            i = int(rng.integers(1, 598))
+            bad[0, h, i], bad[0, h, i + 1] = bad[0, h, i + 1], bad[0, h, i]
+        for i in rng.integers(0, 600, 5):
+            bad[0, h, i] = w.nblk + int(rng.integers(0, 50))
+        for i in rng.integers(1, 600, 5):
+            bad[0, h, i] = bad[0, h, i - 1]
+    got, code = H.gpu_decode(p, 0, q_st, blocks=bad)
+    assert code & lr.LR_DEVERR_BLOCK_ORDER and code & lr.LR_DEVERR_BLOCK_RANGE
+    kept = [[_accepted(list(bad[0, h]), w.nblk) for h in range(w.n_kv_heads)]]
+    assert all(len(k) > 500 for k in kept[0])
+    ref = H.oracle_decode(p, 0, q_ref, blocks=kept)
+    H.assert_attention_close(got, ref)
+
+
 def test_bad_residual_pointers_set_the_error_word():
     w = H.small(T=1000)
     p = H.packed_problem(w)
