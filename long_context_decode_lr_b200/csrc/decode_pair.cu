@@ -85,15 +85,22 @@ constexpr float kGeluC1 = 0.80015708f;  // tanh-form GELU: c1, c3 minimise the l
                                         // against x Phi(x) on [-10, 10] (2.71e-4)
 constexpr float kGeluC3 = 0.03470089f;
 
-__device__ __forceinline__ float gelu_f32(float x) {
-  const float z = x * fmaf(kGeluC3, x * x, kGeluC1);
-  const float h = 0.5f * x;
-  return fmaf(h, tanh_fast(z), h);
-}
-
+// GELU of two GELU-branch inputs: x = u + b1 in fp32, rounded once to fp16 (saturating), then
+// the tanh form evaluated on the fp16 pair (packed half2 arithmetic and the half2 tanh
+// approximation: half the instructions of the fp32 form; the result is stored as fp16 for
+// the next contraction either way).
 __device__ __forceinline__ uint32_t gelu_pair(uint32_t u0, uint32_t u1, uint32_t bias_h2) {
   const float2 bf = __half22float2(*reinterpret_cast<const __half2*>(&bias_h2));
-  return pack_f16x2_sat(gelu_f32(__uint_as_float(u0) + bf.x), gelu_f32(__uint_as_float(u1) + bf.y));
+  const uint32_t xb = pack_f16x2_sat(__uint_as_float(u0) + bf.x, __uint_as_float(u1) + bf.y);
+  const __half2 x = *reinterpret_cast<const __half2*>(&xb);
+  const __half2 z = __hmul2(x, __hfma2(__float2half2_rn(kGeluC3), __hmul2(x, x), __float2half2_rn(kGeluC1)));
+  const uint32_t zb = *reinterpret_cast<const uint32_t*>(&z);
+  uint32_t tb;
+  asm("tanh.approx.f16x2 %0, %1;" : "=r"(tb) : "r"(zb));
+  const __half2 t = *reinterpret_cast<const __half2*>(&tb);
+  const __half2 h = __hmul2(__float2half2_rn(0.5f), x);
+  const __half2 g = __hfma2(h, t, h);
+  return *reinterpret_cast<const uint32_t*>(&g);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
