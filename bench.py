@@ -350,8 +350,8 @@ def decode_launches_per_step(w: synth.Workload, n_sel: int) -> int:
 # roofline.traffic only while that source is unchanged; otherwise traffic is null.
 NCU_TRAFFIC = {
     # prep + pair + combine kernels of one step
-    "llama_262k_full": ("3e3fbe5071b267e3", 2.651e6 + 567.557e6 + 0.457e6 + 2.041e6),
-    "mistral_group_32k": ("3e3fbe5071b267e3", 2.7e6 + 76.9e6 + 0.1e6 + 2.0e6),
+    "llama_262k_full": ("efdfa928c2356715", 2.66e6 + 567.54e6 + 0.23e6 + 2.04e6),
+    "mistral_group_32k": ("efdfa928c2356715", 2.66e6 + 76.99e6 + 0.54e6 + 2.04e6),
 }
 
 
