@@ -35,7 +35,7 @@ def _check(e, k):
         np.testing.assert_array_equal(got[s], ref)
 
 
-@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 1000, 4097])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 1000, 2048, 3001, 4096, 4097])
 @pytest.mark.parametrize("ties", [False, True])
 def test_topk_small(T, ties):
     e = synth.error_vectors(T * 7 + ties, 3, T, ties=ties)
