@@ -255,34 +255,54 @@ fit_grad_kernel(const __grid_constant__ CUtensorMap mapR, const __grid_constant_
 // theta -= lr * scale * sum for every parameter of every weight head; the sums are cleared and
 // the fp16 copies of W1, W_lin, W2 refreshed (update = 0 with lr = 0: only the copies and the
 // clearing, used before the first step). One grid row per weight head (blockIdx.y), so each
-// thread's position within the head's parameters needs no division.
-__device__ __forceinline__ void fit_update_one(const FitUpdateArgs& a, float* w, __half* wh16, void* out, size_t o,
-                                               float d) {
-  const float v = w[o] - d;
-  w[o] = v;
-  if (wh16) wh16[o] = __float2half_rn(v);
-  if (out) store_dtype(out, o, v, a.out_bf16);
+// thread's position within the head's parameters needs no division. Each thread takes
+// kUpdPer parameters of its weight head, strided by the block, and loads
+// all their gradient sums and fp32 masters before it stores anything (a grid of one CTA per
+// 256 parameters left every warp waiting on one load at a time).
+constexpr int kUpdPer = 8;
+
+struct UpdTarget {
+  float* w;
+  __half* wh16;
+  void* out;
+  size_t o;
+};
+
+__device__ __forceinline__ UpdTarget upd_target(const FitUpdateArgs& a, size_t wh, int e) {
+  const int H = a.H, n_wl = 128 * 128, n_w1 = H * 128, n_w2 = 128 * H;
+  if (e < n_wl) return {a.W_lin, a.Wlh, a.out_Wl, wh * n_wl + e};
+  if (e < n_wl + n_w1) return {a.W1, a.W1h, a.out_W1, wh * n_w1 + (e - n_wl)};
+  if (e < n_wl + n_w1 + n_w2) return {a.W2, a.W2h, a.out_W2, wh * n_w2 + (e - n_wl - n_w1)};
+  if (e < n_wl + n_w1 + n_w2 + H) return {a.b1, nullptr, a.out_b1, wh * H + (e - n_wl - n_w1 - n_w2)};
+  return {a.b2, nullptr, a.out_b2, wh * 128 + (e - n_wl - n_w1 - n_w2 - H)};  // b2 may be null
 }
 
-__global__ void fit_update_kernel(FitUpdateArgs a) {
+__global__ void __launch_bounds__(256) fit_update_kernel(FitUpdateArgs a) {
   const size_t wh = blockIdx.y;
-  const int H = a.H;
-  const int n_wl = 128 * 128, n_w1 = H * 128, n_w2 = 128 * H;
   float* g = a.grad + wh * (size_t)a.gstride;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < a.gstride; e += gridDim.x * blockDim.x) {
-    const float d = a.lr * a.scale * g[e];
-    g[e] = 0.f;
-    if (e < n_wl) {
-      fit_update_one(a, a.W_lin, a.Wlh, a.out_Wl, wh * n_wl + e, d);
-    } else if (e < n_wl + n_w1) {
-      fit_update_one(a, a.W1, a.W1h, a.out_W1, wh * n_w1 + (e - n_wl), d);
-    } else if (e < n_wl + n_w1 + n_w2) {
-      fit_update_one(a, a.W2, a.W2h, a.out_W2, wh * n_w2 + (e - n_wl - n_w1), d);
-    } else if (e < n_wl + n_w1 + n_w2 + H) {
-      fit_update_one(a, a.b1, nullptr, a.out_b1, wh * H + (e - n_wl - n_w1 - n_w2), d);
-    } else if (a.b2) {
-      fit_update_one(a, a.b2, nullptr, a.out_b2, wh * 128 + (e - n_wl - n_w1 - n_w2 - H), d);
+  const int e0 = blockIdx.x * (256 * kUpdPer) + threadIdx.x;
+  float gv[kUpdPer], wv[kUpdPer];
+#pragma unroll
+  for (int u = 0; u < kUpdPer; ++u) {
+    const int e = e0 + 256 * u;
+    gv[u] = wv[u] = 0.f;
+    if (e < a.gstride) {
+      const UpdTarget t = upd_target(a, wh, e);
+      gv[u] = g[e];
+      if (t.w) wv[u] = t.w[t.o];
     }
+  }
+#pragma unroll
+  for (int u = 0; u < kUpdPer; ++u) {
+    const int e = e0 + 256 * u;
+    if (e >= a.gstride) break;
+    g[e] = 0.f;
+    const UpdTarget t = upd_target(a, wh, e);
+    if (!t.w) continue;
+    const float v = wv[u] - a.lr * a.scale * gv[u];
+    t.w[t.o] = v;
+    if (t.wh16) t.wh16[t.o] = __float2half_rn(v);
+    if (t.out) store_dtype(t.out, t.o, v, a.out_bf16);
   }
 }
 
@@ -309,7 +329,7 @@ cudaError_t launch_fit_grad(const FitGradArgs& a, const CUtensorMap& mR, const C
 
 cudaError_t launch_fit_update(const FitUpdateArgs& a, cudaStream_t st) {
   if (a.n_heads == 0) return cudaSuccess;
-  fit_update_kernel<<<dim3((a.gstride + 255) / 256, a.n_heads), 256, 0, st>>>(a);
+  fit_update_kernel<<<dim3((a.gstride + 256 * kUpdPer - 1) / (256 * kUpdPer), a.n_heads), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
