@@ -208,10 +208,18 @@ __global__ void __launch_bounds__(SEL_THREADS) select_reduce_kernel(SelectArgs a
   if (x >= n) return;
   const int h = (int)(x % a.Hkv), j = (int)((x / a.Hkv) % a.nblk), b = (int)(x / ((long long)a.nblk * a.Hkv));
   const int G = a.G, P = a.Hkv * G;
+  // every partial sum is loaded before any is added (G <= 8, n_split <= 4)
+  float t[4][8];
+#pragma unroll
+  for (int z = 0; z < 4; ++z)
+#pragma unroll
+    for (int g = 0; g < 8; ++g)
+      t[z][g] = (z < a.n_split && g < G) ? a.partial[(((size_t)z * a.B + b) * a.nblk + j) * P + h * G + g] : 0.f;
   float m = -CUDART_INF_F;
-  for (int g = 0; g < G; ++g) {
-    float v = 0.f;
-    for (int z = 0; z < a.n_split; ++z) v += a.partial[(((size_t)z * a.B + b) * a.nblk + j) * P + h * G + g];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    if (g >= G) break;
+    const float v = ((t[0][g] + t[1][g]) + t[2][g]) + t[3][g];
     m = g == 0 ? v : fmaxf(m, v);
   }
   a.scores[((size_t)b * a.Hkv + h) * a.nblk + j] = m;
