@@ -34,6 +34,15 @@
  *     word gets LR_DEVERR_TIMEOUT).
  *   - The last failing host-side check's message is available, per thread, from
  *     lr_last_error().
+ *   - Kernel families: decode calls on bf16 caches with hd = 128, H of 128 or 256,
+ *     r a multiple of 64 and at most 8 query heads per KV head, and lr_pack_prefill
+ *     on bf16 with hd = 128, H of 128 or 256 and r a multiple of 128, run on the
+ *     tensor-core kernels; other shapes run on CUDA-core kernels, with the same
+ *     results to the stated tolerances. Two
+ *     environment variables, read at each call, force the CUDA-core kernels on
+ *     shapes the tensor-core kernels would take: LOWRAM_DECODE_PATH=general (decode
+ *     entry points) and LOWRAM_PACK_PATH=general (lr_pack_prefill). Any other value,
+ *     or none, keeps the default choice. They exist for testing and comparison.
  *
  * Notation: B batch (sequences), T context tokens, L_g layers per group,
  * Hkv KV heads, G = Hq / Hkv query heads per KV head (query head hq reads KV
